@@ -1,0 +1,152 @@
+/*
+ * cowa.h -- C ABI of libcowa.so: CoWindow Attention (CoWA) on NVIDIA B200 (sm_100a).
+ *
+ * What the operation is.  CoWA ("CoWindow Attention: Full Causal Coverage Is a
+ * Collective Property", Abstract; skillfed.io news summary of 2026-09-30,
+ * paragraphs 2, 4, 6 and 7) is exact softmax attention under a mask that is a
+ * function of positions and of the global KV-head index only.  For KV head g
+ * (global index G = kv_head_base + g, H = h_kv_global KV heads in the layer)
+ * a query at position t sees key s iff s <= t and one of:
+ *   - s is in the shared prefix sink      [0, S)
+ *   - s is in the shared near-diagonal    (t-L, t]        (L >= 1 keys incl. t)
+ *   - s is in G's long-range interval     [b_p, b_{p+1}),  b_i = S + floor(i*(T-S)/H),
+ *                                                          p = (G mod D) * (H/D)
+ * With D = H the H intervals partition [S, T) and the union over KV heads is
+ * the whole causal prefix; D < H repeats D distinct intervals over the heads
+ * (the duplicated-window ablation, news summary paragraph 3).  L >= T gives
+ * dense causal attention (the FullAttn comparison of the Abstract).  The
+ * interval formula and the D < H slot rule are this library's reading: the
+ * pages state the principle, not a formula.
+ *
+ * Query head h uses KV head g = h / (H_q / H_kv) (grouped-query attention).
+ * Each head applies its softmax over its own visible keys (news summary,
+ * paragraph 7).  Scores are softmax_scale * q.k; lse is the natural log of
+ * the softmax denominator.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are bf16 in device memory, described by cowa_tensor: a pointer
+ *     plus element strides for batch, position and head; the head dimension d
+ *     is contiguous.  Pointers and every stride * 2 bytes must be multiples
+ *     of 16 bytes (COWA_ERR_ALIGNMENT otherwise).  d must be 64 or 128
+ *     (COWA_ERR_UNSUPPORTED otherwise).
+ *   - The caller owns every buffer, including the workspace; the library never
+ *     allocates device memory on a call.  Query the workspace size with the
+ *     matching *_workspace_size function; a smaller ws_bytes returns
+ *     COWA_ERR_WORKSPACE.  The workspace must be 256-byte aligned.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Argument errors are returned before any
+ *     launch; a failed launch returns COWA_ERR_CUDA.  No exception crosses the
+ *     ABI.  Outputs are deterministic (no atomics in any result).
+ *   - Device-side waits are bounded: a wait that runs out sets a status word
+ *     in the workspace and the kernel returns; cowa_workspace_status() reads
+ *     it (COWA_ERR_TIMEOUT).
+ *   - The library keeps no mutable global state on the call path; calls on
+ *     different streams with different workspaces may run concurrently.
+ */
+#ifndef COWA_H
+#define COWA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  COWA_OK = 0,
+  COWA_ERR_INVALID_ARG = 1, /* bad shape, pattern or null pointer */
+  COWA_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128} */
+  COWA_ERR_ALIGNMENT = 3,   /* pointer or stride not 16-byte aligned */
+  COWA_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
+  COWA_ERR_CUDA = 5,        /* CUDA runtime/driver error at launch */
+  COWA_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out */
+} cowa_status;
+
+/* Window parameters of one attention layer.
+ *   S  prefix-sink size, 0 <= S <= T
+ *   L  near-diagonal width in keys (includes the query's own key), L >= 1
+ *   T  declared span: the long-range region is [S, T); T >= S
+ *   D  number of distinct long-range intervals, 1 <= D, D divides h_kv_global
+ *   kv_head_base  global index of this call's KV head 0 (0 on one GPU; KV-head
+ *                 tensor parallelism passes r * H / P on rank r)
+ *   h_kv_global   H, KV heads in the whole layer (0 means "= H_kv of the call")
+ *   softmax_scale multiplier of q.k (<= 0 means 1/sqrt(d)) */
+typedef struct {
+  int32_t S, L, T, D;
+  int32_t kv_head_base;
+  int32_t h_kv_global;
+  float softmax_scale;
+} cowa_pattern;
+
+/* A bf16 device tensor with the head dimension contiguous.  Element (b, t, h, :)
+ * starts at ptr + b*stride_b + t*stride_t + h*stride_h (strides in elements).
+ * [B, N, H, d] contiguous has stride_t = H*d, stride_h = d, stride_b = N*H*d. */
+typedef struct {
+  void* ptr;
+  int64_t stride_b, stride_t, stride_h;
+} cowa_tensor;
+
+/* ---- forward (training / prefill self-attention at positions 0..N-1) ------------------
+ * Inputs  q [B, N, H_q, d], k and v [B, N, H_kv, d]   (bf16, cowa_tensor strides)
+ * Outputs o [B, N, H_q, d] bf16; lse fp32, contiguous [B, H_q, N] (natural log), saved
+ *         for cowa_bwd.
+ * H_q must be a multiple of H_kv.  N >= 1. */
+size_t cowa_fwd_workspace_size(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d);
+cowa_status cowa_fwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d,
+                     cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, float* lse,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---- backward ---------------------------------------------------------------------------
+ * Gradients of sum(dO * O) for the forward above, from the saved o and lse.
+ * Inputs  q, k, v, o, lse as produced/consumed by cowa_fwd; dO [B, N, H_q, d] bf16.
+ * Outputs dq [B, N, H_q, d], dk and dv [B, N, H_kv, d], bf16 (fp32 accumulation).
+ * The workspace holds fp32 row statistics and fp32 gradient accumulators. */
+size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d);
+cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d,
+                     cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse,
+                     cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---- decode (one new token per sequence, KV cache) -----------------------------------------
+ * q_t    [B, H_q, d] bf16, contiguous.
+ * k_cache, v_cache: cowa_tensor over [B, T_cap, H_kv, d]-indexed (b, t, h) with any strides
+ *        (e.g. [B, H_kv, T_cap, d] has stride_h = T_cap*d, stride_t = d).
+ * pos    device int32 [B]: the new token's position; its own K/V are already written at
+ *        pos[b]; 0 <= pos[b] < T_cap (entries outside are clamped into range).
+ * o      [B, H_q, d] bf16 contiguous; lse_or_null fp32 [B, H_q] or NULL.
+ * Reads only the cache rows the pattern makes visible at pos[b]. */
+size_t cowa_decode_workspace_size(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap);
+cowa_status cowa_decode(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap,
+                        const void* q_t, cowa_tensor k_cache, cowa_tensor v_cache,
+                        const int32_t* pos, void* o, float* lse_or_null,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---- status --------------------------------------------------------------------------------
+ * Synchronizes `stream`, reads and clears the device status word in `ws` (the workspace of an
+ * earlier call), and returns COWA_OK or COWA_ERR_TIMEOUT (COWA_ERR_CUDA if the stream failed). */
+cowa_status cowa_workspace_status(void* ws, void* stream);
+const char* cowa_status_string(cowa_status s);
+
+/* ---- planner introspection (host; tests and tools) -----------------------------------------
+ * The same integer code the kernels run.
+ * cowa_visible_counts: out[g*N + t] = number of keys visible to position t for local KV head g
+ *   (host memory, H_kv*N int64).
+ * cowa_plan_debug: writes records of the tile plan for tile sizes BM x BN into host `out`:
+ *   which = 0  forward plan, records (g, i, j, full) for every visited (q-tile i, kv-tile j)
+ *   which = 1  backward plan, records (g, j, i, 0) for every q-tile i that sees kv-tile j
+ *   which = 2  forward plan evaluated by a device kernel (same records in arbitrary order;
+ *              `out` is still host memory, `dev_scratch` must be device memory of at least
+ *              256 + cap*16 bytes; the call synchronizes the device)
+ *   Records are 4 int32 each, in (g, outer, inner) order.  *n_written receives the number of
+ *   records; if it exceeds cap, only cap are written and COWA_ERR_WORKSPACE is returned. */
+cowa_status cowa_visible_counts(const cowa_pattern* pat, int H_kv, int N, int64_t* out);
+cowa_status cowa_plan_debug(const cowa_pattern* pat, int H_kv, int N, int BM, int BN, int which,
+                            int32_t* out, size_t cap, size_t* n_written, void* dev_scratch);
+
+int cowa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COWA_H */

@@ -230,31 +230,48 @@ def _row_visible_cols(t: int, pat: Pattern, g: int, h_kv: int) -> np.ndarray:
     return np.nonzero(m)[0]
 
 
-def attention_fwd_rows(q, k, v, pat: Pattern, rows, b: int, heads=None):
+def attention_fwd_rows(q, k, v, pat: Pattern, rows, b: int, heads=None, block: int = 256):
     """o[len(rows), len(heads), d] and lse[len(rows), len(heads)] at query positions `rows` of batch b.
 
-    q/k/v may be any array-likes indexable as [b, t, h, :] (e.g. float64 arrays).
+    Rows are evaluated in runs of consecutive positions (at most `block` long):
+    for each run and KV head the explicit mask is built over [0, t_max], the
+    columns that any row of the run sees are gathered once, and each row's
+    softmax runs over its own masked scores.  q/k/v may be any array-likes
+    indexable as [b, t, h, :] / [b, cols, g, :] that convert to float64.
     """
     Hq = q.shape[2]; Hkv = k.shape[2]; d = q.shape[3]
     grp = Hq // Hkv
     heads = list(range(Hq)) if heads is None else list(heads)
     scale = pat.sm_scale(d)
+    rows = np.asarray(rows, dtype=np.int64)
     o = np.zeros((len(rows), len(heads), d))
     lse = np.zeros((len(rows), len(heads)))
-    for ri, t in enumerate(rows):
-        cache = {}
-        for hi_, h in enumerate(heads):
-            g = h // grp
-            if g not in cache:
-                cols = _row_visible_cols(int(t), pat, g, Hkv)
-                cache[g] = (np.asarray(k[b, cols, g, :], np.float64), np.asarray(v[b, cols, g, :], np.float64))
-            kk, vv = cache[g]
-            sc = scale * (kk @ np.asarray(q[b, t, h, :], np.float64))
-            m = sc.max()
-            e = np.exp(sc - m)
-            den = e.sum()
-            lse[ri, hi_] = m + math.log(den)
-            o[ri, hi_] = (e / den) @ vv
+    order = np.argsort(rows, kind="stable")
+    srt = rows[order]
+    # runs of consecutive sorted positions
+    starts = [0] + [i for i in range(1, len(srt)) if srt[i] != srt[i - 1] + 1 or i % block == 0]
+    bounds = list(zip(starts, starts[1:] + [len(srt)]))
+    by_g = {}
+    for hi_, h in enumerate(heads):
+        by_g.setdefault(h // grp, []).append((hi_, h))
+    for a0, a1 in bounds:
+        run = srt[a0:a1]
+        idx = order[a0:a1]
+        tmax = int(run[-1])
+        for g, hs in by_g.items():
+            m = visible_mask(run, tmax + 1, pat, g, Hkv)
+            cols = np.nonzero(m.any(axis=0))[0]
+            mm = m[:, cols]
+            kk = np.asarray(k[b, cols, g, :], np.float64)
+            vv = np.asarray(v[b, cols, g, :], np.float64)
+            for hi_, h in hs:
+                qh = np.asarray(q[b, run, h, :], np.float64)
+                sc = np.where(mm, scale * (qh @ kk.T), -np.inf)
+                mx = sc.max(axis=1, keepdims=True)
+                e = np.exp(sc - mx)
+                den = e.sum(axis=1, keepdims=True)
+                lse[idx, hi_] = (mx + np.log(den))[:, 0]
+                o[idx, hi_] = (e / den) @ vv
     return o, lse
 
 

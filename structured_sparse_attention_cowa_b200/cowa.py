@@ -1,0 +1,255 @@
+"""Python binding of libcowa.so: argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+turns torch tensors into the C ABI's pointers and strides, allocates the
+caller-owned outputs and workspace with torch, and raises on any non-OK
+status.  There is no fallback: if libcowa.so is missing or fails to load,
+every call raises.
+
+Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_bwd,
+cowa_decode, plus the planner introspection helpers.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcowa.so")
+
+COWA_OK = 0
+_STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED", 3: "COWA_ERR_ALIGNMENT",
+           4: "COWA_ERR_WORKSPACE", 5: "COWA_ERR_CUDA", 6: "COWA_ERR_TIMEOUT"}
+
+EXPORTED = ["cowa_fwd_workspace_size", "cowa_fwd", "cowa_bwd_workspace_size", "cowa_bwd",
+            "cowa_decode_workspace_size", "cowa_decode", "cowa_workspace_status", "cowa_status_string",
+            "cowa_visible_counts", "cowa_plan_debug", "cowa_version"]
+
+
+class CowaError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {_STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+class c_pattern(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int32), ("L", ctypes.c_int32), ("T", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("kv_head_base", ctypes.c_int32), ("h_kv_global", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+class c_tensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride_b", ctypes.c_int64), ("stride_t", ctypes.c_int64),
+                ("stride_h", ctypes.c_int64)]
+
+
+@dataclasses.dataclass(frozen=True)
+class Pattern:
+    """CoWA window parameters (see include/cowa.h, cowa_pattern)."""
+
+    S: int
+    L: int
+    T: int
+    D: int
+    kv_head_base: int = 0
+    h_kv_global: int = 0
+    softmax_scale: float = 0.0
+
+    def c(self) -> c_pattern:
+        return c_pattern(self.S, self.L, self.T, self.D, self.kv_head_base, self.h_kv_global, self.softmax_scale)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcowa.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libcowa.so not found at {LIB_PATH}; build it with "
+                           "`python -m structured_sparse_attention_cowa_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, T, vp, i, sz = ctypes.POINTER(c_pattern), c_tensor, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.cowa_fwd_workspace_size.argtypes = [P, i, i, i, i, i]
+    L.cowa_fwd_workspace_size.restype = sz
+    L.cowa_fwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, vp, sz, vp]
+    L.cowa_fwd.restype = i
+    L.cowa_bwd_workspace_size.argtypes = [P, i, i, i, i, i]
+    L.cowa_bwd_workspace_size.restype = sz
+    L.cowa_bwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
+    L.cowa_bwd.restype = i
+    L.cowa_decode_workspace_size.argtypes = [P, i, i, i, i, i]
+    L.cowa_decode_workspace_size.restype = sz
+    L.cowa_decode.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp, sz, vp]
+    L.cowa_decode.restype = i
+    L.cowa_workspace_status.argtypes = [vp, vp]
+    L.cowa_workspace_status.restype = i
+    L.cowa_status_string.argtypes = [i]
+    L.cowa_status_string.restype = ctypes.c_char_p
+    L.cowa_visible_counts.argtypes = [P, i, i, vp]
+    L.cowa_visible_counts.restype = i
+    L.cowa_plan_debug.argtypes = [P, i, i, i, i, i, vp, sz, ctypes.POINTER(sz), vp]
+    L.cowa_plan_debug.restype = i
+    L.cowa_version.argtypes = []
+    L.cowa_version.restype = i
+    _lib = L
+    return L
+
+
+def _check(fn: str, status: int):
+    if status != COWA_OK:
+        raise CowaError(fn, status, lib().cowa_status_string(status).decode())
+
+
+def _t4(x) -> c_tensor:
+    """[B, N, H, d] tensor (d contiguous) -> cowa_tensor."""
+    if x.dim() != 4 or x.stride(3) != 1:
+        raise ValueError("expected a [B, N, H, d] tensor with the last dim contiguous")
+    return c_tensor(x.data_ptr(), x.stride(0), x.stride(1), x.stride(2))
+
+
+def _stream(stream):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _workspace(nbytes: int, device):
+    import torch
+
+    return torch.zeros(max(256, nbytes), dtype=torch.uint8, device=device)
+
+
+def _bf16_cuda(name, x):
+    import torch
+
+    if not (x.is_cuda and x.dtype == torch.bfloat16):
+        raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+
+
+def cowa_fwd(q, k, v, pattern: Pattern, out=None, lse=None, workspace=None, stream=None):
+    """o [B,N,H_q,d] bf16 and lse [B,H_q,N] fp32 of CoWA attention over q, k, v."""
+    import torch
+
+    for n_, x_ in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n_, x_)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_fwd_workspace_size(ctypes.byref(pat), B, N, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q.device)
+    _check("cowa_fwd", L.cowa_fwd(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v), _t4(out),
+                                  lse.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """(dq, dk, dv) bf16: gradients of sum(do * o) for the forward with the same inputs."""
+    import torch
+
+    for n_, x_ in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _bf16_cuda(n_, x_)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_bwd_workspace_size(ctypes.byref(pat), B, N, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q.device)
+    _check("cowa_bwd", L.cowa_bwd(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v), _t4(o),
+                                  lse.data_ptr(), _t4(do), _t4(dq), _t4(dk), _t4(dv),
+                                  workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def _cache_tensor(x, layout: str) -> c_tensor:
+    if x.dim() != 4 or x.stride(3) != 1:
+        raise ValueError("cache must be 4-D with the head dim contiguous")
+    if layout == "bhtd":   # [B, H_kv, T_cap, d]
+        return c_tensor(x.data_ptr(), x.stride(0), x.stride(2), x.stride(1))
+    if layout == "bthd":   # [B, T_cap, H_kv, d]
+        return c_tensor(x.data_ptr(), x.stride(0), x.stride(1), x.stride(2))
+    raise ValueError("layout must be 'bhtd' or 'bthd'")
+
+
+def cowa_decode(q_t, k_cache, v_cache, pos, pattern: Pattern, layout: str = "bhtd", out=None, lse=None,
+                workspace=None, stream=None, want_lse: bool = True):
+    """o [B,H_q,d] bf16 (and lse [B,H_q] fp32) for one new token per sequence at pos[b]."""
+    import torch
+
+    for n_, x_ in (("q_t", q_t), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _bf16_cuda(n_, x_)
+    B, Hq, d = q_t.shape
+    if layout == "bhtd":
+        Hkv, T_cap = k_cache.shape[1], k_cache.shape[2]
+    else:
+        T_cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if not q_t.is_contiguous():
+        raise ValueError("q_t must be contiguous [B, H_q, d]")
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise TypeError("pos must be a CUDA int32 tensor [B]")
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_t.device) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_t.device)
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_decode_workspace_size(ctypes.byref(pat), B, Hq, Hkv, d, T_cap)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q_t.device)
+    _check("cowa_decode", L.cowa_decode(ctypes.byref(pat), B, Hq, Hkv, d, T_cap, q_t.data_ptr(),
+                                        _cache_tensor(k_cache, layout), _cache_tensor(v_cache, layout),
+                                        pos.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
+                                        workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def workspace_status(workspace, stream=None) -> int:
+    """Read (and clear) the device status word of a workspace; returns the cowa_status code."""
+    return lib().cowa_workspace_status(ctypes.c_void_p(workspace.data_ptr()), _stream(stream))
+
+
+# ---------------------------------------------------------------------------- introspection
+def visible_counts(pattern: Pattern, h_kv: int, N: int) -> np.ndarray:
+    out = np.zeros((h_kv, N), dtype=np.int64)
+    pat = pattern.c()
+    _check("cowa_visible_counts", lib().cowa_visible_counts(ctypes.byref(pat), h_kv, N,
+                                                            out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def plan_debug(pattern: Pattern, h_kv: int, N: int, BM: int, BN: int, which: int, dev_scratch=None) -> np.ndarray:
+    """Tile-plan records, int32 [n, 4]; which = 0 fwd (host), 1 bwd (host), 2 fwd (device kernel)."""
+    pat = pattern.c()
+    L = lib()
+    n = ctypes.c_size_t(0)
+    cap = 1024
+    while True:
+        out = np.zeros((cap, 4), dtype=np.int32)
+        scratch = None
+        if which == 2:
+            import torch
+
+            scratch = torch.zeros(256 + cap * 16, dtype=torch.uint8, device="cuda") if dev_scratch is None else dev_scratch
+        st = L.cowa_plan_debug(ctypes.byref(pat), h_kv, N, BM, BN, which, out.ctypes.data_as(ctypes.c_void_p), cap,
+                               ctypes.byref(n), ctypes.c_void_p(scratch.data_ptr()) if scratch is not None else None)
+        if st == 4 and n.value > cap:
+            cap = int(n.value)
+            continue
+        _check("cowa_plan_debug", st)
+        return out[: n.value].copy()

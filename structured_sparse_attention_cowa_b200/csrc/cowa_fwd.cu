@@ -1,0 +1,386 @@
+// cowa_fwd.cu -- CoWA forward on sm_100a: exact softmax attention over the position-defined
+// visible set of each KV head ("CoWindow Attention: Full Causal Coverage Is a Collective
+// Property", Abstract; skillfed.io news summary, paragraphs 2 and 7).
+//
+// One CTA = (batch b, KV head g, 128-row query tile i, a pair of query heads of g's GQA
+// group).  The two heads share every K/V tile the CTA loads and the same tile plan, because
+// the mask depends on g only.  Warp roles (10 warps):
+//   warps 0-3  softmax for head slot 0 (thread = query row = TMEM lane)
+//   warps 4-7  softmax for head slot 1
+//   warp  8    TMA producer: Q once, then K_j, V_j of every visited KV tile into a 3-deep ring
+//   warp  9    tcgen05 MMA issuer (one lane): S = Q K^T into TMEM, O += P V into TMEM
+// The visited KV tiles come from the planner (sink tiles, interval_g tiles, near-diagonal
+// band, merged); only tiles that are not entirely visible apply the element mask.
+// Online softmax in the log2 domain with a lazy rescale of O (only when the running max
+// grows by more than 2^8), P rounded to bf16 into a 128-byte-swizzled shared tile, fp32
+// accumulation throughout.  Epilogue: O / l -> bf16 o, lse = ln(sum exp) in fp32.
+//
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "cowa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace cowa {
+namespace {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kFwdThreads = 320;
+constexpr int kRing = 3;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdGeom {
+  static constexpr int kQBytes = kBM * D * 2;     // one head's Q tile
+  static constexpr int kKVBytes = kBN * D * 2;    // one K or V tile
+  static constexpr int kPBytes = kBM * kBN * 2;   // one head's P tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kQBytes;
+  static constexpr int kOffP = kOffRing + kRing * kKVBytes;
+  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;  // + alignment slack
+  static constexpr int kColO = 256;
+};
+
+struct Tiles {
+  Range r[3];
+  int n;     // number of ranges
+  int count; // number of tiles
+};
+
+__device__ __forceinline__ Tiles plan_tiles(const Pat& p, Range iv, int t0, int t1) {
+  Tiles T;
+  T.n = fwd_tile_ranges(p, iv, t0, t1, kBN, T.r);
+  T.count = 0;
+  for (int x = 0; x < T.n; ++x) T.count += T.r[x].hi - T.r[x].lo;
+  return T;
+}
+
+// Walks the tile list in order.
+struct TileCursor {
+  int x, j;
+  __device__ __forceinline__ void init(const Tiles& T) { x = 0; j = T.n > 0 ? T.r[0].lo : 0; }
+  __device__ __forceinline__ void next(const Tiles& T) {
+    if (++j >= T.r[x].hi && x + 1 < T.n) { ++x; j = T.r[x].lo; }
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_constant__ FwdArgs a) {
+  using Geo = FwdGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t kv_full[kRing], kv_empty[kRing];
+  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_ready[2], o_done[2];
+  __shared__ __align__(8) uint64_t mma_final;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: heaviest (last) query tiles first; all heads/pairs of one tile adjacent
+  const int grp = a.Hq / a.Hkv;
+  const int npair = (grp + 1) >> 1;
+  const int nq = (a.N + kBM - 1) / kBM;
+  const int per_i = a.B * a.Hkv * npair;
+  const int i = nq - 1 - (int)(blockIdx.x / per_i);
+  int rem = blockIdx.x % per_i;
+  const int pair = rem % npair; rem /= npair;
+  const int g = rem % a.Hkv;
+  const int b = rem / a.Hkv;
+  const int h0 = g * grp + 2 * pair;
+  const bool has1 = (2 * pair + 1) < grp;
+  const int t0 = i * kBM, t1 = imin(a.N, t0 + kBM);
+  const Range iv = interval_of(a.pat, g);
+  const Tiles T = plan_tiles(a.pat, iv, t0, t1);
+
+  uint8_t* sQ = smem + Geo::kOffQ;
+  uint8_t* sRing = smem + Geo::kOffRing;
+  uint8_t* sP = smem + Geo::kOffP;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&q_full, 1);
+    for (int s = 0; s < kRing; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
+    for (int k = 0; k < 2; ++k) {
+      ptx::mbar_init(&s_full[k], 1);
+      ptx::mbar_init(&s_free[k], 4);
+      ptx::mbar_init(&p_ready[k], 4);
+      ptx::mbar_init(&o_done[k], 1);
+    }
+    ptx::mbar_init(&mma_final, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(&tmem_base_sh, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const int ntiles = T.count;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&a.tm_q);
+      ptx::tma_prefetch_desc(&a.tm_k);
+      ptx::tma_prefetch_desc(&a.tm_v);
+      ptx::mbar_arrive_expect_tx(&q_full, (has1 ? 2 : 1) * Geo::kQBytes);
+      for (int u = 0; u < D / 64; ++u) {
+        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, t0, h0, b);
+        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, t0, h0 + 1, b);
+      }
+      TileCursor cur;
+      cur.init(T);
+      int issued = 0;
+      for (int idx = 0; idx < 2 * ntiles; ++idx) {
+        const int s = idx % kRing;
+        if (idx >= kRing && !ptx::mbar_wait(&kv_empty[s], ((idx / kRing) - 1) & 1, &abort_flag, a.status)) break;
+        const bool is_v = idx & 1;
+        uint8_t* dst = sRing + s * Geo::kKVBytes;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], Geo::kKVBytes);
+        for (int u = 0; u < D / 64; ++u)
+          ptx::tma_load_4d(dst + u * 16384, is_v ? &a.tm_v : &a.tm_k, &kv_full[s], u * 64, cur.j * kBN, g, b);
+        if (is_v) cur.next(T);
+        issued = idx + 1;
+      }
+      // drain: no copy may still be landing in shared memory when the CTA exits
+      ptx::mbar_wait(&q_full, 0, nullptr, a.status);
+      for (int idx = (issued > kRing ? issued - kRing : 0); idx < issued; ++idx)
+        ptx::mbar_wait(&kv_full[idx % kRing], (idx / kRing) & 1, nullptr, a.status);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+      const uint32_t q_addr = ptx::smem_u32(sQ), ring_addr = ptx::smem_u32(sRing), p_addr = ptx::smem_u32(sP);
+      const int nslot = has1 ? 2 : 1;
+
+      auto issue_s = [&](int k, int kslot) {
+        const uint32_t qa = q_addr + k * Geo::kQBytes, kb = ring_addr + kslot * Geo::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + k * 128, ptx::smem_desc_sw128(qa + off, 16, 1024),
+                           ptx::smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int k, int vslot, bool accumulate) {
+        const uint32_t pa = p_addr + k * Geo::kPBytes, vb = ring_addr + vslot * Geo::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + Geo::kColO + k * D, ptx::smem_desc_sw128(pa + aoff, 16, 1024),
+                           ptx::smem_desc_sw128(vb + kk * 2048, 16384, 1024), idesc_o,
+                           (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
+      ptx::tc_fence_after();
+      for (int n = 0; ok && n < ntiles; ++n) {
+        const int kidx = 2 * n, vidx = 2 * n + 1;
+        const int kslot = kidx % kRing, vslot = vidx % kRing;
+        if (!(ok = ptx::mbar_wait(&kv_full[kslot], (kidx / kRing) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        // S0(n)
+        if (n > 0 && !(ok = ptx::mbar_wait(&s_free[0], (n - 1) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        issue_s(0, kslot);
+        ptx::mma_commit(&s_full[0]);
+        if (nslot == 2) {
+          // PV1(n-1): overlaps with softmax 0 working on S0(n)
+          if (n > 0) {
+            const int pv = 2 * (n - 1) + 1;
+            if (!(ok = ptx::mbar_wait(&p_ready[1], (n - 1) & 1, &abort_flag, a.status))) break;
+            ptx::tc_fence_after();
+            issue_pv(1, pv % kRing, n - 1 > 0);
+            ptx::mma_commit(&o_done[1]);
+            ptx::mma_commit(&kv_empty[pv % kRing]);
+          }
+          // S1(n)
+          if (n > 0 && !(ok = ptx::mbar_wait(&s_free[1], (n - 1) & 1, &abort_flag, a.status))) break;
+          ptx::tc_fence_after();
+          issue_s(1, kslot);
+          ptx::mma_commit(&s_full[1]);
+        }
+        ptx::mma_commit(&kv_empty[kslot]);
+        // PV0(n)
+        if (!(ok = ptx::mbar_wait(&kv_full[vslot], (vidx / kRing) & 1, &abort_flag, a.status))) break;
+        if (!(ok = ptx::mbar_wait(&p_ready[0], n & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        issue_pv(0, vslot, n > 0);
+        ptx::mma_commit(&o_done[0]);
+        if (nslot == 1) ptx::mma_commit(&kv_empty[vslot]);
+      }
+      if (ok && nslot == 2 && ntiles > 0) {
+        const int n = ntiles - 1, pv = 2 * n + 1;
+        if (ptx::mbar_wait(&p_ready[1], n & 1, &abort_flag, a.status)) {
+          ptx::tc_fence_after();
+          issue_pv(1, pv % kRing, n > 0);
+          ptx::mma_commit(&o_done[1]);
+          ptx::mma_commit(&kv_empty[pv % kRing]);
+        }
+      }
+      // all issued MMAs complete before TMEM can be released
+      ptx::mma_commit(&mma_final);
+      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int k = warp >> 2;  // head slot
+    if (k == 0 || has1) {
+      const int r = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
+      const int t = t0 + r;
+      const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      const uint32_t s_tm = lane_base + k * 128;
+      const uint32_t o_tm = lane_base + Geo::kColO + k * D;
+      uint8_t* prow = sP + k * Geo::kPBytes + r * 128;
+      float m_used = -INFINITY, l = 0.f;
+      const float sl2 = a.scale_log2;
+      bool ok = true;
+      TileCursor cur;
+      cur.init(T);
+      for (int n = 0; n < ntiles; ++n, cur.next(T)) {
+        const int s0 = cur.j * kBN;
+        const bool need_mask = (s0 + kBN > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kBN));
+        if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_tm + c * 32, sr + c * 32);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&s_free[k]);
+
+        float x[128];
+        float mx = -INFINITY;
+        if (need_mask) {
+          // visible key columns of row t within [s0, s0+128), relative to s0
+          const int sink_end = imin(a.pat.S, t + 1) - s0;
+          const int band_lo = imax(0, t - a.pat.L + 1) - s0;
+          const int diag_end = t + 1 - s0;
+          const int lr_lo = iv.lo - s0, lr_hi = imin(iv.hi, t + 1) - s0;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const bool vis = (c < sink_end) || (c >= band_lo && c < diag_end) || (c >= lr_lo && c < lr_hi);
+            x[c] = vis ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
+            mx = fmaxf(mx, x[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            x[c] = __uint_as_float(sr[c]) * sl2;
+            mx = fmaxf(mx, x[c]);
+          }
+        }
+        const float m_new = fmaxf(m_used, mx);
+        // the previous PV of this head must be done before P is overwritten / O rescaled
+        if (n > 0 && !(ok = ptx::mbar_wait_warp(&o_done[k], (n - 1) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        // lazy rescale: only when the running max grows by more than 2^8 (or first finite max)
+        const bool grow = (m_new != -INFINITY) && (m_used == -INFINITY || m_new > m_used + kRescaleThreshold);
+        float alpha = 1.f;
+        if (grow) {
+          alpha = ptx::ex2(m_used - m_new);  // 0 when nothing was visible before
+          l *= alpha;
+          m_used = m_new;
+        }
+        if (n > 0 && __any_sync(0xffffffffu, grow)) {
+          // O row *= alpha, a warp-collective TMEM round trip (alpha = 1 on the other lanes)
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(o_tm + c * 32, ov);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            ptx::tmem_st32(o_tm + c * 32, ov);
+          }
+          ptx::tmem_wait_st();
+        }
+        const float m_eff = m_used == -INFINITY ? 0.f : m_used;
+        float rowsum = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 16; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ptx::ex2(x[c8 * 8 + 2 * e] - m_eff);
+            const float p1 = ptx::ex2(x[c8 * 8 + 2 * e + 1] - m_eff);
+            rowsum += p0 + p1;
+            w[e] = ptx::pack_bf16(p0, p1);
+          }
+          const int chunk = c8 >> 3, unit = c8 & 7;
+          uint4* dst = reinterpret_cast<uint4*>(prow + chunk * 16384 + ((unit ^ (r & 7)) << 4));
+          *dst = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l += rowsum;
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&p_ready[k]);
+      }
+      // ---- epilogue
+      if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], (ntiles - 1) & 1, &abort_flag, a.status)) {
+        ptx::tc_fence_after();
+        uint32_t ov[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(o_tm + c * 32, ov + c * 32);
+        ptx::tmem_wait_ld();
+        if (t < a.N) {
+          const float inv = 1.f / l;
+          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)t * a.o_st +
+                                (size_t)(h0 + k) * a.o_sh;
+#pragma unroll
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = ptx::pack_bf16(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv,
+                                    __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv);
+            reinterpret_cast<uint4*>(orow)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          a.lse[((size_t)b * a.Hq + h0 + k) * a.N + t] = (m_used + log2f(l)) * 0.69314718055994530942f;
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
+  using Geo = FwdGeom<D>;
+  auto kern = cowa_fwd_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  const int grp = a.Hq / a.Hkv;
+  const int nq = (a.N + kBM - 1) / kBM;
+  const long long nblk = (long long)nq * a.B * a.Hkv * ((grp + 1) / 2);
+  if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
+  kern<<<(unsigned)nblk, kFwdThreads, Geo::kSmem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s) {
+  if (a.d == 64) return launch_fwd_d<64>(a, s);
+  if (a.d == 128) return launch_fwd_d<128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cowa

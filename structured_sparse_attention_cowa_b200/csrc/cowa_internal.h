@@ -1,0 +1,80 @@
+// cowa_internal.h -- declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/cowa.h"
+#include "cowa_pattern.h"
+
+namespace cowa {
+
+// Every workspace starts with a 256-byte header whose first word is the device
+// status (0 = ok, bit 0 = a bounded wait ran out).  Kernel data follows.
+constexpr size_t kWsHeader = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Encode a 4-D bf16 tensor map over (d, t, h, b) with a box of (64, box_rows, 1, 1)
+// and 128-byte swizzle.  Returns false if the driver rejects it.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n_t, int n_h, int n_b, int64_t stride_t,
+                    int64_t stride_h, int64_t stride_b, int box_rows);
+
+// ---- decode ----
+struct DecodeArgs {
+  Pat pat;
+  int B, Hq, Hkv, d, T_cap;
+  const void* q_t;
+  const int32_t* pos;
+  void* o;
+  float* lse;        // may be null
+  float* partials;   // [B, Hq, n_split, d + 2]
+  uint32_t* status;
+  int chunk;         // tokens per split
+  int n_split;
+  float scale_log2;  // softmax scale * log2(e)
+  CUtensorMap tm_k, tm_v;
+};
+int decode_chunk_tokens(const Pat& p, int B, int Hkv, int T_cap);
+int decode_num_splits(const Pat& p, int T_cap, int chunk);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+// ---- forward ----
+struct FwdArgs {
+  Pat pat;
+  int B, N, Hq, Hkv, d;
+  void* o;
+  int64_t o_sb, o_st, o_sh;
+  float* lse;
+  uint32_t* status;
+  float scale_log2;
+  CUtensorMap tm_q, tm_k, tm_v;
+};
+cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s);
+
+// ---- backward ----
+struct BwdArgs {
+  Pat pat;
+  int B, N, Hq, Hkv, d;
+  const void* o; int64_t o_sb, o_st, o_sh;
+  const void* dO; int64_t do_sb, do_st, do_sh;
+  const float* lse;
+  void* dq; int64_t dq_sb, dq_st, dq_sh;
+  void* dk; int64_t dk_sb, dk_st, dk_sh;
+  void* dv; int64_t dv_sb, dv_st, dv_sh;
+  float* delta;      // [B, Hq, N] fp32 workspace
+  uint32_t* status;
+  float scale;       // softmax scale
+  float scale_log2;  // softmax scale * log2(e)
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+};
+size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d);
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t s);
+
+// ---- planner debug kernel ----
+cudaError_t launch_plan_debug(const Pat& p, int Hkv, int N, int BM, int BN, int32_t* dev_out, size_t cap,
+                              unsigned long long* dev_count, cudaStream_t s);
+
+}  // namespace cowa

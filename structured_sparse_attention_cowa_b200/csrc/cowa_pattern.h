@@ -1,0 +1,134 @@
+// cowa_pattern.h -- CoWA visibility pattern and tile planner as plain integer arithmetic.
+//
+// Used unchanged by the host (validation, introspection) and by every kernel
+// (on the fly, per CTA).  The pattern is a function of positions and of the
+// global KV-head index only ("CoWindow Attention: Full Causal Coverage Is a
+// Collective Property", Abstract: no learned router or indexer; skillfed.io
+// news summary, paragraphs 2 and 4).
+//
+//   visible(t, s, G) = s <= t  and  ( s < S  or  s > t - L  or  s in I_G )
+//   I_G = [b_p, b_{p+1}),  b_i = S + floor(i*(T-S)/H),  p = (G mod D) * (H/D)
+//
+// Everything here returns half-open ranges [lo, hi) and never touches memory.
+#pragma once
+
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define COWA_HD __host__ __device__ __forceinline__
+#else
+#define COWA_HD inline
+#endif
+
+namespace cowa {
+
+struct Pat {
+  int S, L, T, D;
+  int G0;  // global index of local KV head 0
+  int H;   // KV heads in the layer
+};
+
+struct Range {
+  int lo, hi;  // [lo, hi); empty if lo >= hi
+};
+
+COWA_HD int imin(int a, int b) { return a < b ? a : b; }
+COWA_HD int imax(int a, int b) { return a > b ? a : b; }
+
+// b_i = S + floor(i * (T - S) / H), in 64-bit to avoid overflow of i*(T-S).
+COWA_HD int bound(const Pat& p, int i) {
+  return p.S + (int)(((int64_t)i * (int64_t)(p.T - p.S)) / (int64_t)p.H);
+}
+
+// Long-range interval of local KV head g.
+COWA_HD Range interval_of(const Pat& p, int g) {
+  const int G = p.G0 + g;
+  const int slot = (G % p.D) * (p.H / p.D);
+  return Range{bound(p, slot), bound(p, slot + 1)};
+}
+
+COWA_HD bool visible(const Pat& p, Range iv, int t, int s) {
+  return s <= t && (s < p.S || s > t - p.L || (s >= iv.lo && s < iv.hi));
+}
+
+// Sort up to three ranges by lo, drop empty ones and merge overlapping or
+// touching ones.  Returns the number of disjoint ranges written to r[0..n).
+COWA_HD int merge3(Range a, Range b, Range c, Range* r) {
+  Range v[3] = {a, b, c};
+  // 3-element sorting network on lo (empty ranges pushed last by lo = INT_MAX)
+  for (int i = 0; i < 3; ++i)
+    if (v[i].lo >= v[i].hi) { v[i].lo = 0x7fffffff; v[i].hi = 0x7fffffff; }
+  if (v[1].lo < v[0].lo) { Range x = v[0]; v[0] = v[1]; v[1] = x; }
+  if (v[2].lo < v[1].lo) { Range x = v[1]; v[1] = v[2]; v[2] = x; }
+  if (v[1].lo < v[0].lo) { Range x = v[0]; v[0] = v[1]; v[1] = x; }
+  int n = 0;
+  for (int i = 0; i < 3; ++i) {
+    if (v[i].lo == 0x7fffffff) break;
+    if (n > 0 && v[i].lo <= r[n - 1].hi) {
+      r[n - 1].hi = imax(r[n - 1].hi, v[i].hi);
+    } else {
+      r[n++] = v[i];
+    }
+  }
+  return n;
+}
+
+// Keys visible to position t (local KV head g, interval iv), as <= 3 disjoint
+// sorted ranges: sink [0, min(S, t+1)), band [max(0, t-L+1), t+1), and
+// interval [lo, min(hi, t+1)).
+COWA_HD int row_ranges(const Pat& p, Range iv, int t, Range* r) {
+  Range sink{0, imin(p.S, t + 1)};
+  Range band{imax(0, t - p.L + 1), t + 1};
+  Range lr{iv.lo, imin(iv.hi, t + 1)};
+  return merge3(sink, band, lr, r);
+}
+
+// Forward plan: KV tiles (of BN keys) that rows [t0, t1) visit, as <= 3
+// disjoint sorted tile-index ranges.  Exactly the tiles whose block holds at
+// least one visible element: the union over t in [t0, t1) of the row ranges
+// is sink [0, min(S, t1)), band [max(0, t0-L+1), t1), interval [lo, min(hi, t1)).
+COWA_HD int fwd_tile_ranges(const Pat& p, Range iv, int t0, int t1, int BN, Range* r) {
+  Range sink{0, imin(p.S, t1)};
+  Range band{imax(0, t0 - p.L + 1), t1};
+  Range lr{iv.lo, imin(iv.hi, t1)};
+  Range tk[3];
+  const Range src[3] = {sink, band, lr};
+  for (int i = 0; i < 3; ++i) {
+    if (src[i].lo < src[i].hi) {
+      tk[i].lo = src[i].lo / BN;
+      tk[i].hi = (src[i].hi + BN - 1) / BN;
+    } else {
+      tk[i].lo = 0; tk[i].hi = 0;
+    }
+  }
+  return merge3(tk[0], tk[1], tk[2], r);
+}
+
+// True iff every (t, s) with t in [t0, t1), s in [s0, s1) is visible.
+// Requires s1 - 1 <= t0 (all keys at or before every query); the hardest row
+// is t1 - 1, whose band starts latest, so [s0, s1) must lie inside
+// [0, S) U I_g U [t1 - L, inf).
+COWA_HD bool tile_full(const Pat& p, Range iv, int t0, int t1, int s0, int s1) {
+  if (s1 - 1 > t0) return false;
+  int x = s0;
+  // walk right through the covering segments; at most three steps
+  for (int it = 0; it < 4 && x < s1; ++it) {
+    if (x < p.S) { x = p.S; continue; }
+    if (x >= iv.lo && x < iv.hi) { x = iv.hi; continue; }
+    if (x >= t1 - p.L) { x = s1; continue; }
+    return false;
+  }
+  return x >= s1;
+}
+
+// Backward plan: the rows that see any key of [s0, s1) form one contiguous
+// range starting at s0: a sink or interval key s is seen by every t >= s, a
+// band-only key s by t in [s, s+L).  Returns rows [s0, end) clipped to N.
+COWA_HD Range bwd_row_range(const Pat& p, Range iv, int s0, int s1, int N) {
+  // smallest key of the tile that is in the sink or the interval
+  bool special = (s0 < p.S) || (iv.lo < iv.hi && iv.lo < s1 && iv.hi > s0);
+  int end = special ? N : imin(N, s1 - 1 + p.L);
+  return Range{s0, imax(s0, end)};
+}
+
+}  // namespace cowa

@@ -1,0 +1,151 @@
+"""Host-side checks of libcowa.so: it loads, exports every function include/cowa.h declares,
+its planner matches the oracle's mask-derived plan bit for bit, and bad arguments return
+the documented status before any launch.  No GPU is touched here."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import cowa_oracle as orc
+from structured_sparse_attention_cowa_b200 import cowa as cw
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    txt = open(os.path.join(ROOT, "include", "cowa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(cowa_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = cw.lib()
+    names = _declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.cowa_version() >= 1
+
+
+def _oracle_pattern(p: cw.Pattern):
+    return orc.Pattern(S=p.S, L=p.L, T=p.T, D=p.D, kv_head_base=p.kv_head_base,
+                       h_kv_global=p.h_kv_global or None)
+
+
+PLAN_CASES = [
+    # N, Hkv, BM, BN, pattern
+    (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 4)),       # tiny config
+    (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 2)),       # duplicated D=2
+    (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 1)),       # duplicated D=1
+    (1000, 4, 128, 128, cw.Pattern(64, 128, 1000, 4)),       # ragged tail
+    (777, 3, 64, 32, cw.Pattern(0, 1, 700, 3)),              # no sink, L=1, N > T
+    (600, 2, 128, 128, cw.Pattern(130, 70, 600, 2)),         # sink not tile aligned
+    (512, 4, 128, 128, cw.Pattern(16, 512, 512, 4)),         # dense causal (L >= T)
+    (300, 4, 32, 32, cw.Pattern(4, 60, 4, 1)),               # SWA + sinks (T = S)
+    (257, 2, 128, 128, cw.Pattern(3, 9, 257, 2, kv_head_base=2, h_kv_global=4)),  # TP rank
+]
+
+
+@pytest.mark.parametrize("N,Hkv,BM,BN,pat", PLAN_CASES)
+def test_host_plans_match_mask_bit_exact(N, Hkv, BM, BN, pat):
+    op = _oracle_pattern(pat)
+    fwd = cw.plan_debug(pat, Hkv, N, BM, BN, 0)
+    want = sorted((g, i, j, int(full)) for (i, g), lst in orc.tile_plan_fwd(N, BM, BN, op, Hkv).items()
+                  for j, full in lst)
+    assert sorted(map(tuple, fwd.tolist())) == want
+    bwd = cw.plan_debug(pat, Hkv, N, BM, BN, 1)
+    want_b = sorted((g, j, i, 0) for (j, g), lst in orc.tile_plan_bwd(N, BM, BN, op, Hkv).items() for i in lst)
+    assert sorted(map(tuple, bwd.tolist())) == want_b
+
+
+@pytest.mark.parametrize("N,Hkv,BM,BN,pat", PLAN_CASES)
+def test_visible_counts_bit_exact(N, Hkv, BM, BN, pat):
+    got = cw.visible_counts(pat, Hkv, N)
+    want = orc.visible_counts(N, _oracle_pattern(pat), Hkv)
+    assert np.array_equal(got, want)
+
+
+def _closed_form_counts(N, S, L, T, H, D, g):
+    """|sink U band U interval| per position by inclusion-exclusion (vectorised over t)."""
+    b = [S + (i * (T - S)) // H for i in range(H + 1)]
+    p = (g % D) * (H // D)
+    lo, hi = b[p], b[p + 1]
+    t = np.arange(N, dtype=np.int64)
+    def inter(a0, a1, b0, b1):
+        return np.maximum(0, np.minimum(a1, b1) - np.maximum(a0, b0))
+    A = (np.zeros_like(t), np.minimum(S, t + 1))
+    Bd = (np.maximum(0, t - L + 1), t + 1)
+    C = (np.full_like(t, lo), np.minimum(hi, t + 1))
+    n = lambda r: np.maximum(0, r[1] - r[0])
+    ab = inter(*A, *Bd); ac = inter(*A, *C); bc = inter(*Bd, *C)
+    abc = np.maximum(0, np.minimum(np.minimum(A[1], Bd[1]), C[1]) - np.maximum(np.maximum(A[0], Bd[0]), C[0]))
+    return n(A) + n(Bd) + n(C) - ab - ac - bc + abc
+
+
+@pytest.mark.parametrize("N,S,L,T,H,D", [(32768, 128, 2048, 32768, 8, 8), (131072, 128, 4096, 131072, 8, 8),
+                                          (8192, 128, 1024, 8192, 8, 2)])
+def test_visible_counts_of_the_long_configs(N, S, L, T, H, D):
+    """Host planner counts at the 8K / 32K / 128K shapes against a closed form, and the union
+    over heads covers the causal prefix."""
+    pat = cw.Pattern(S, L, T, D)
+    c = cw.visible_counts(pat, H, N)
+    for g in range(H):
+        assert np.array_equal(c[g], _closed_form_counts(N, S, L, T, H, D, g))
+    if D == H:
+        assert (c.sum(0) >= np.arange(1, N + 1)).all()
+
+
+# ---------------------------------------------------------------------------- validation
+def _t(ptr=0x10000, sb=1 << 20, st=1024, sh=128):
+    return cw.c_tensor(ptr, sb, st, sh)
+
+
+def _fwd(pat, B=1, N=128, Hq=8, Hkv=4, d=128, q=None, lse=0x20000, ws=0x40000, ws_bytes=1 << 20):
+    p = pat.c() if pat is not None else None
+    return cw.lib().cowa_fwd(ctypes.byref(p) if p is not None else None, B, N, Hq, Hkv, d, q or _t(), _t(), _t(),
+                             _t(), lse, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(pat=None), 1),
+    (dict(pat=cw.Pattern(64, 0, 1024, 4)), 1),          # L = 0
+    (dict(pat=cw.Pattern(64, 8, 32, 4)), 1),            # T < S
+    (dict(pat=cw.Pattern(64, 8, 1024, 3)), 1),          # D does not divide H
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), Hq=6), 1),    # Hq % Hkv
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), d=96), 2),    # head dim
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), Hq=40, Hkv=4), 2),  # group of 10 > 8
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), q=cw.c_tensor(0x10008, 1 << 20, 1024, 128)), 3),  # misaligned ptr
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), q=cw.c_tensor(0x10000, 1 << 20, 1020, 128)), 3),  # misaligned stride
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), q=cw.c_tensor(0, 1 << 20, 1024, 128)), 1),        # null
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), lse=0), 1),
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), ws_bytes=16), 4),
+    (dict(pat=cw.Pattern(64, 8, 1024, 4), ws=0x40010), 4),  # workspace not 256-aligned
+    (dict(pat=cw.Pattern(64, 8, 1024, 4, kv_head_base=2, h_kv_global=4)), 1),  # base + Hkv > H
+])
+def test_fwd_rejects_bad_arguments_before_launch(kwargs, status):
+    assert _fwd(**kwargs) == status
+
+
+def test_decode_and_bwd_reject_bad_arguments():
+    L = cw.lib()
+    p = cw.Pattern(64, 8, 1024, 4).c()
+    # decode: null pos
+    assert L.cowa_decode(ctypes.byref(p), 2, 8, 4, 128, 1024, 0x10000, _t(), _t(), None, 0x30000, None,
+                         0x40000, 1 << 20, None) == 1
+    # decode: small workspace
+    assert L.cowa_decode(ctypes.byref(p), 2, 8, 4, 128, 1024, 0x10000, _t(), _t(), 0x50000, 0x30000, None,
+                         0x40000, 8, None) == 4
+    # bwd: misaligned dO
+    assert L.cowa_bwd(ctypes.byref(p), 1, 128, 8, 4, 128, _t(), _t(), _t(), _t(), 0x20000,
+                      cw.c_tensor(0x10004, 1 << 20, 1024, 128), _t(), _t(), _t(), 0x40000, 1 << 30, None) == 3
+    assert L.cowa_fwd_workspace_size(ctypes.byref(p), 1, 128, 8, 4, 96) == 0
+    assert L.cowa_decode_workspace_size(ctypes.byref(p), 16, 40, 8, 128, 131072) > 0
+
+
+def test_status_strings():
+    L = cw.lib()
+    for s in range(7):
+        assert len(L.cowa_status_string(s)) > 0
