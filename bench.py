@@ -1,0 +1,468 @@
+"""Benchmark of the CoWA hot path on B200: one step = cowa_fwd + cowa_bwd on the 32K
+training layer plus cowa_decode on the 128K decode cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cowa|reference]
+
+Prints one JSON line (rank 0).  `value` is visible TFLOP/s of the training part
+(forward 4*d and backward 10*d FLOPs per visible query-key pair, summed over all
+ranks) divided by the max-over-ranks device time of the whole step (decode
+included); `parts` gives each call's CUDA-event time, the decode GB/s over the
+visible K/V bytes, and the same for the dense-causal mode when --dense is given.
+Inputs are larger than L2 (126 MB), so no flush is needed between steps.
+
+N > 1: one process per GPU (torchrun); every rank runs the same per-GPU workload on
+its own batch element and seeds (weak scaling: batch sharding, no exchange step in
+the op), timed between barriers, max over ranks.
+
+--impl reference times the CPU fp64 oracle (test infrastructure, not the product) on a
+bounded sample of the same workload, on the host cores of rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CoWA fwd/bwd TFLOP/s (visible) + decode GB/s at 32K/128K, % of B200 roofline"
+
+# Train 32K layer (B=1 per GPU) and decode 128K cache (B=16 per GPU)
+TRAIN = dict(B=1, N=32768, Hq=40, Hkv=8, d=128, S=128, L=2048, T=32768, D=8)
+DECODE = dict(B=16, Hq=40, Hkv=8, d=128, T_cap=131072, S=128, L=4096, T=131072, D=8, pos=131071)
+
+
+# ------------------------------------------------------------------------------ accounting
+def visible_pairs(N, S, L, T, D, Hkv, Hq, B=1, h_kv_global=None):
+    """Sum over b, query heads and positions of |visible keys| (closed form per position)."""
+    import numpy as np
+
+    H = h_kv_global or Hkv
+    grp = Hq // Hkv
+    bnd = [S + (i * (T - S)) // H for i in range(H + 1)]
+    t = np.arange(N, dtype=np.int64)
+    total = 0
+    for g in range(Hkv):
+        p = (g % D) * (H // D)
+        lo, hi = bnd[p], bnd[p + 1]
+        sink = np.minimum(S, t + 1)
+        band_lo = np.maximum(0, t - L + 1)
+        band = t + 1 - band_lo
+        lr_hi = np.minimum(hi, t + 1)
+        lr = np.maximum(0, lr_hi - lo)
+        sb = np.maximum(0, np.minimum(S, t + 1) - band_lo)               # sink & band
+        lb = np.maximum(0, lr_hi - np.maximum(lo, band_lo))              # interval & band
+        ls = np.maximum(0, np.minimum(S, lr_hi) - lo)                    # interval & sink (0: lo >= S)
+        total += int((sink + band + lr - sb - lb - ls).sum())
+    return total * grp * B
+
+
+def decode_visible_tokens(pos, S, L, T, D, Hkv, h_kv_global=None):
+    H = h_kv_global or Hkv
+    bnd = [S + (i * (T - S)) // H for i in range(H + 1)]
+    out = []
+    for g in range(Hkv):
+        p = (g % D) * (H // D)
+        lo, hi = bnd[p], bnd[p + 1]
+        ranges = sorted([(0, min(S, pos + 1)), (max(0, pos - L + 1), pos + 1), (lo, min(hi, pos + 1))])
+        n, cur = 0, None
+        for a, b in ranges:
+            if a >= b:
+                continue
+            if cur is None or a > cur[1]:
+                if cur:
+                    n += cur[1] - cur[0]
+                cur = [a, b]
+            else:
+                cur[1] = max(cur[1], b)
+        n += cur[1] - cur[0]
+        out.append(n)
+    return out
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return pk["bf16_tflops"], pk["bf16_tflops_sustained"], pk["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _traffic_record(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    src = os.path.join(ROOT, "structured_sparse_attention_cowa_b200", "csrc", kernel_file)
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        for line in open(path):
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == kernel_file and parts[1] == sha:
+                return float(parts[2])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"cowa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                sm.append(float(p[1]))
+                mx = float(p[2])
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        except Exception:
+            return None
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+_KV_CACHE = {}
+
+
+def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
+    """Time the fp64 oracle forward on row blocks of the 32K config until ~target_s of CPU work
+    (input generation is outside the timed part).  Returns (visible TFLOP/s, description,
+    threads, seconds timed)."""
+    import numpy as np
+
+    from oracle import cowa_oracle as orc
+    from structured_sparse_attention_cowa_b200 import synth
+
+    c = TRAIN
+    pat = orc.Pattern(S=c["S"], L=c["L"], T=c["T"], D=c["D"])
+    rng = np.random.default_rng(99)
+    Hkv, Hq, d, N = c["Hkv"], c["Hq"], c["d"], c["N"]
+
+    class Rows:
+        """A seeded bf16 tensor widened to float64 on access (the oracle reads slices)."""
+
+        def __init__(self, name, H):
+            self.bits = synth.normal_bf16_bits((1, N, H, d), synth.seed_of(name, seed_extra))
+            self.shape = self.bits.shape
+
+        def __getitem__(self, idx):
+            return orc.bf16_bits_to_f64(self.bits[idx])
+
+    if seed_extra not in _KV_CACHE:
+        _KV_CACHE[seed_extra] = (Rows("k", Hkv), Rows("v", Hkv))
+    k, v = _KV_CACHE[seed_extra]
+
+    class QRows:
+        """Query rows drawn per 32-row block (only the sampled rows are ever generated)."""
+
+        shape = (1, N, Hq, d)
+
+        def __getitem__(self, idx):
+            b, rows, h, _ = idx
+            rows = np.atleast_1d(rows)
+            blk = synth.normal_bf16_bits((len(rows), d), synth.seed_of("q", seed_extra) + 7919 * int(rows[0]) + h)
+            return orc.bf16_bits_to_f64(blk)
+
+    q = QRows()
+    done_flops, t_used, nblocks = 0.0, 0.0, 0
+    while t_used < target_s and nblocks < 512:
+        t0 = int(rng.integers(0, N - 32))
+        rows = np.arange(t0, t0 + 32)
+        st = time.perf_counter()
+        orc.attention_fwd_rows(q, k, v, pat, rows, b=0)
+        t_used += time.perf_counter() - st
+        pairs = 0
+        for g in range(Hkv):
+            pairs += int(orc.visible_mask(rows, int(rows[-1]) + 1, pat, g, Hkv).sum()) * (Hq // Hkv)
+        done_flops += 4.0 * d * pairs
+        nblocks += 1
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = (f"oracle forward (fp64 numpy, explicit mask) on {nblocks} random 32-row blocks x {Hq} heads "
+            f"of the 32K layer, visible FLOPs credited")
+    return done_flops / t_used / 1e12, desc, threads, t_used
+
+
+# ------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cowa", choices=["cowa", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dense", action="store_true", help="also time the dense-causal mode (L >= T)")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_cowa(args, world, rank, local)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    per = max(1.0, min(20.0, 120.0 / (steps + warm)))
+    vals = []
+    for i in range(warm + steps):
+        v, desc, threads, used = cpu_oracle_sample(per, seed_extra=i % 3)
+        if i >= warm:
+            vals.append((v, used))
+    value = statistics.median(v for v, _ in vals)
+    ms = statistics.mean(u for _, u in vals) * 1e3
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "train 32K layer, oracle forward on row samples", **TRAIN},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_cowa(args, world, rank, local):
+    import torch
+
+    from structured_sparse_attention_cowa_b200 import cowa as cw
+    from structured_sparse_attention_cowa_b200 import synth
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c, dc = TRAIN, DECODE
+    pat = cw.Pattern(c["S"], c["L"], c["T"], c["D"])
+    pat_dense = cw.Pattern(c["S"], c["N"], c["T"], c["D"])
+    dpat = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
+
+    # ---- inputs (per rank: its own batch element / seeds), outputs, workspaces
+    ex = rank
+    q = synth.cuda_normal_bf16((c["B"], c["N"], c["Hq"], c["d"]), synth.seed_of("q", ex), dev)
+    k = synth.cuda_normal_bf16((c["B"], c["N"], c["Hkv"], c["d"]), synth.seed_of("k", ex), dev)
+    v = synth.cuda_normal_bf16((c["B"], c["N"], c["Hkv"], c["d"]), synth.seed_of("v", ex), dev)
+    do = synth.cuda_normal_bf16((c["B"], c["N"], c["Hq"], c["d"]), synth.seed_of("do", ex), dev)
+    kc = synth.cuda_normal_bf16((dc["B"], dc["Hkv"], dc["T_cap"], dc["d"]), synth.seed_of("k_cache", ex), dev)
+    vc = synth.cuda_normal_bf16((dc["B"], dc["Hkv"], dc["T_cap"], dc["d"]), synth.seed_of("v_cache", ex), dev)
+    qt = synth.cuda_normal_bf16((dc["B"], dc["Hq"], dc["d"]), synth.seed_of("q_t", ex), dev)
+    pos = torch.full((dc["B"],), dc["pos"], dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((c["B"], c["Hq"], c["N"]), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    od = torch.empty((dc["B"], dc["Hq"], dc["d"]), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((dc["B"], dc["Hq"]), dtype=torch.float32, device=dev)
+    import ctypes
+
+    L = cw.lib()
+    cp = pat.c()
+    cpd = dpat.c()
+    ws_f = torch.zeros(max(256, L.cowa_fwd_workspace_size(ctypes.byref(cp), c["B"], c["N"], c["Hq"], c["Hkv"], c["d"])),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.zeros(L.cowa_bwd_workspace_size(ctypes.byref(cp), c["B"], c["N"], c["Hq"], c["Hkv"], c["d"]),
+                       dtype=torch.uint8, device=dev)
+    ws_d = torch.zeros(L.cowa_decode_workspace_size(ctypes.byref(cpd), dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                    dc["T_cap"]), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        cw.cowa_fwd(q, k, v, pat, out=o, lse=lse, workspace=ws_f)
+
+    def bwd():
+        cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+
+    def dec():
+        cw.cowa_decode(qt, kc, vc, pos, dpat, out=od, lse=lsed, workspace=ws_d)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def maxr(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- warm-up
+    for _ in range(max(3, args.warmup)):
+        fwd(); bwd(); dec()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, events between the three calls
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e_start.record()
+        for s in range(K):
+            ev[s][0].record(); fwd(); ev[s][1].record(); bwd(); ev[s][2].record(); dec(); ev[s][3].record()
+        e_end.record()
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = maxr(e_start.elapsed_time(e_end))
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    dec_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    for st in (cw.workspace_status(ws_f), cw.workspace_status(ws_b), cw.workspace_status(ws_d)):
+        if st != 0:
+            raise RuntimeError(f"device status {st} after the timed region")
+
+    pairs = visible_pairs(c["N"], c["S"], c["L"], c["T"], c["D"], c["Hkv"], c["Hq"], c["B"])
+    fwd_flop = 4.0 * c["d"] * pairs
+    bwd_flop = 10.0 * c["d"] * pairs
+    toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
+    dec_bytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2  # K and V rows, bf16
+    ms_step = total_ms / K
+    value = world * (fwd_flop + bwd_flop) / (ms_step * 1e-3) / 1e12
+
+    burst, sustained, hbm, peak_src = _peaks()
+    parts = {
+        "fwd": {"ms": fwd_ms, "tflops_visible": fwd_flop / (fwd_ms * 1e-3) / 1e12},
+        "bwd": {"ms": bwd_ms, "tflops_visible": bwd_flop / (bwd_ms * 1e-3) / 1e12},
+        "decode": {"ms": dec_ms, "gbs_visible": dec_bytes / (dec_ms * 1e-3) / 1e9,
+                   "frac_hbm": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "visible_bytes": dec_bytes},
+    }
+    for p in ("fwd", "bwd"):
+        parts[p]["frac_peak"] = parts[p]["tflops_visible"] / sustained
+
+    # ---- dense-causal mode (FullAttn comparison), optional
+    if args.dense:
+        def fwd_d():
+            cw.cowa_fwd(q, k, v, pat_dense, out=o, lse=lse, workspace=ws_f)
+        fwd_d(); torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(3):
+            fwd_d()
+        b.record(); torch.cuda.synchronize()
+        dms = a.elapsed_time(b) / 3
+        dpairs = c["N"] * (c["N"] + 1) // 2 * c["Hq"] * c["B"]
+        parts["fwd_dense_causal"] = {"ms": dms, "tflops": 4.0 * c["d"] * dpairs / (dms * 1e-3) / 1e12,
+                                     "speedup_cowa_vs_dense": dms / fwd_ms}
+
+    # ---- roofline of the dominant kernel: the forward kernel is one launch per cowa_fwd
+    fwd_traffic = _traffic_record("cowa_fwd.cu")
+    roofline = {"kernel": "cowa_fwd_kernel<128>", "bound": "tensor", "achieved": parts["fwd"]["tflops_visible"],
+                "peak": sustained, "unit": "TFLOP/s", "frac": parts["fwd"]["tflops_visible"] / sustained,
+                "traffic": fwd_traffic, "peak_source": f"{peak_src} bf16 sustained",
+                "algorithmic": f"{fwd_flop:.4e} FLOP per launch = 4*d*visible pairs ({pairs:.4e})"}
+
+    # ---- end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h_in = [pin(x) for x in (q, k, v, do, qt)]
+        for hsrc, dsrc in zip(h_in, (q, k, v, do, qt)):
+            hsrc.copy_(dsrc)
+        h_pos = pos.cpu().pin_memory()
+        h_out = [pin(x) for x in (o, dq, dk, dv, od)]
+        h2d = sum(x.numel() * x.element_size() for x in h_in) + h_pos.numel() * 4
+        d2h = sum(x.numel() * x.element_size() for x in h_out)
+        KE = max(1, min(K, 3))
+
+        def e2e_step():
+            for hsrc, ddst in zip(h_in, (q, k, v, do, qt)):
+                ddst.copy_(hsrc, non_blocking=True)
+            pos.copy_(h_pos, non_blocking=True)
+            fwd(); bwd(); dec()
+            for ddst, hsrc in zip(h_out, (o, dq, dk, dv, od)):
+                ddst.copy_(hsrc, non_blocking=True)
+
+        e2e_step(); torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(KE):
+            e2e_step()
+        b.record(); torch.cuda.synchronize()
+        barrier()
+        e_ms = maxr(a.elapsed_time(b)) / KE
+        e2e = {"value": world * (fwd_flop + bwd_flop) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE}
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v_cpu, desc, threads, _ = cpu_oracle_sample(args.cpu_seconds)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "host_cpus": os.cpu_count()}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "train 32K layer fwd+bwd + decode 128K cache, per GPU",
+                       "train": TRAIN, "decode": DECODE, "l2": "inputs larger than L2 (126 MB); no flush",
+                       "parallelism": f"batch-sharded x{world} (weak)"},
+            "parts": parts, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": K * 6, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -66,6 +66,7 @@ __all__ = [
     "attention_fwd",
     "attention_bwd",
     "attention_fwd_rows",
+    "attention_bwd_rows",
     "attention_bwd_cols",
     "decode",
     "tile_plan_fwd",
@@ -275,45 +276,89 @@ def attention_fwd_rows(q, k, v, pat: Pattern, rows, b: int, heads=None, block: i
     return o, lse
 
 
+def _block_visible(run, pat, g, Hkv):
+    """Mask rows `run` x the columns any of them sees, and those column indices."""
+    tmax = int(run[-1])
+    m = visible_mask(run, tmax + 1, pat, g, Hkv)
+    cols = np.nonzero(m.any(axis=0))[0]
+    return m[:, cols], cols
+
+
+def attention_bwd_rows(q, k, v, do, pat: Pattern, rows, b: int, heads=None, block: int = 256):
+    """dq[len(rows), len(heads), d] at query positions `rows` of batch b (row-local).
+
+    For each row: P over its visible keys, O = P v, Delta = dO.O, dS = P (dO v^T - Delta),
+    dq = scale dS k.  Consecutive rows are evaluated together as in attention_fwd_rows.
+    """
+    Hq = q.shape[2]; Hkv = k.shape[2]; d = q.shape[3]
+    grp = Hq // Hkv
+    heads = list(range(Hq)) if heads is None else list(heads)
+    scale = pat.sm_scale(d)
+    rows = np.asarray(rows, dtype=np.int64)
+    dq = np.zeros((len(rows), len(heads), d))
+    order = np.argsort(rows, kind="stable")
+    srt = rows[order]
+    starts = [0] + [i for i in range(1, len(srt)) if srt[i] != srt[i - 1] + 1 or i % block == 0]
+    by_g = {}
+    for hi_, h in enumerate(heads):
+        by_g.setdefault(h // grp, []).append((hi_, h))
+    for a0, a1 in zip(starts, starts[1:] + [len(srt)]):
+        run = srt[a0:a1]
+        idx = order[a0:a1]
+        for g, hs in by_g.items():
+            mm, cols = _block_visible(run, pat, g, Hkv)
+            kk = np.asarray(k[b, cols, g, :], np.float64)
+            vv = np.asarray(v[b, cols, g, :], np.float64)
+            for hi_, h in hs:
+                qh = np.asarray(q[b, run, h, :], np.float64)
+                doh = np.asarray(do[b, run, h, :], np.float64)
+                sc = np.where(mm, scale * (qh @ kk.T), -np.inf)
+                e = np.exp(sc - sc.max(axis=1, keepdims=True))
+                P = e / e.sum(axis=1, keepdims=True)
+                O = P @ vv
+                delta = (doh * O).sum(axis=1, keepdims=True)
+                dS = P * (doh @ vv.T - delta)
+                dq[idx, hi_] = scale * (dS @ kk)
+    return dq
+
+
 def attention_bwd_cols(q, k, v, do, pat: Pattern, b: int, g: int, cols, row_block: int = 512):
     """dk_g[cols], dv_g[cols] (local KV head g, batch b) from every row that sees those columns.
 
     Rows that see column s are found from the explicit mask; their softmax
-    statistics (lse, Delta = rowsum(dO*O)) are recomputed here from scratch.
+    statistics (lse, Delta = rowsum(dO*O)) are recomputed here from scratch over
+    each row's own visible keys.
     """
     Hq = q.shape[2]; Hkv = k.shape[2]; d = q.shape[3]; N = q.shape[1]
     grp = Hq // Hkv
     scale = pat.sm_scale(d)
     cols = np.asarray(cols, dtype=np.int64)
-    smin = int(cols.min())
-    kg = np.asarray(k[b, :, g, :], np.float64)
-    vg = np.asarray(v[b, :, g, :], np.float64)
     dk = np.zeros((len(cols), d)); dv = np.zeros((len(cols), d))
-    kc = kg[cols]; vc = vg[cols]
-    for r0 in range(smin, N, row_block):
-        rows = np.arange(r0, min(N, r0 + row_block))
-        # which rows of this block see any of the requested columns
-        msub = visible_mask(rows, N, pat, g, Hkv)
-        seen = msub[:, cols]
-        keep = seen.any(axis=1)
-        if not keep.any():
-            continue
-        rows = rows[keep]; msub = msub[keep]; seen = seen[keep]
+    kc = np.asarray(k[b, cols, g, :], np.float64); vc = np.asarray(v[b, cols, g, :], np.float64)
+    # rows that see at least one requested column
+    seen_rows = np.zeros(N, bool)
+    for s in cols:
+        t = np.arange(s, N)
+        seen_rows[t[visible_mask(t, s + 1, pat, g, Hkv)[:, s]]] = True
+    rows_all = np.nonzero(seen_rows)[0]
+    for r0 in range(0, len(rows_all), row_block):
+        run = rows_all[r0:r0 + row_block]
+        mm, vcols = _block_visible(run, pat, g, Hkv)
+        kk = np.asarray(k[b, vcols, g, :], np.float64)
+        vv = np.asarray(v[b, vcols, g, :], np.float64)
+        seen = visible_mask(run, N, pat, g, Hkv)[:, cols]
         for h in range(g * grp, (g + 1) * grp):
-            qh = np.asarray(q[b, rows, h, :], np.float64)
-            doh = np.asarray(do[b, rows, h, :], np.float64)
-            sc = scale * (qh @ kg[: rows.max() + 1].T)
-            sc = np.where(msub[:, : rows.max() + 1], sc, -np.inf)
+            qh = np.asarray(q[b, run, h, :], np.float64)
+            doh = np.asarray(do[b, run, h, :], np.float64)
+            sc = np.where(mm, scale * (qh @ kk.T), -np.inf)
             m = sc.max(axis=1, keepdims=True)
             e = np.exp(sc - m)
             den = e.sum(axis=1, keepdims=True)
-            P = e / den
-            O = P @ vg[: rows.max() + 1]
+            O = (e / den) @ vv
             delta = (doh * O).sum(axis=1, keepdims=True)
             # P at the requested columns: exp(score - lse) where visible, else 0
             Pc = np.where(seen, np.exp(scale * (qh @ kc.T) - (m + np.log(den))), 0.0)
-            dPc = doh @ vc.T
-            dSc = Pc * (dPc - delta)
+            dSc = Pc * (doh @ vc.T - delta)
             dv += Pc.T @ doh
             dk += scale * (dSc.T @ qh)
     return dk, dv

@@ -229,7 +229,9 @@ cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int
   a.dk = dk.ptr; a.dk_sb = dk.stride_b; a.dk_st = dk.stride_t; a.dk_sh = dk.stride_h;
   a.dv = dv.ptr; a.dv_sb = dv.stride_b; a.dv_st = dv.stride_t; a.dv_sh = dv.stride_h;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.N_pad = (N + 127) / 128 * 128;
   a.delta = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.lse2 = a.delta + (size_t)B * Hq * a.N_pad;
   a.scale = scale_of(pat, d);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   if (!make_tmap_bf16(&a.tm_q, q.ptr, d, N, Hq, B, q.stride_t, q.stride_h, q.stride_b, 128) ||

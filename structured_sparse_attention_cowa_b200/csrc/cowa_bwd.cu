@@ -1,5 +1,522 @@
+// cowa_bwd.cu -- CoWA backward on sm_100a: gradients of exact softmax attention over the
+// position-defined visible set ("CoWindow Attention: Full Causal Coverage Is a Collective
+// Property", Abstract: forward and backward latency of the operator during training).
+//
+// With P = exp(scale * q.k - lse) on visible pairs (0 elsewhere), dP = dO v^T,
+// Delta = rowsum(dO * O) and dS = P * (dP - Delta):
+//   dV_g = sum_h P^T dO_h,   dK_g = scale * sum_h dS^T Q_h,   dQ_h = scale * dS K_g.
+// Three kernels, no atomics (results are deterministic):
+//   1. preprocess: Delta and lse*log2(e) per row into the workspace, padded to whole tiles
+//      (padded rows get lse = +inf so they contribute P = 0);
+//   2. dK/dV: one CTA per (b, KV head g, 128-key tile j); K_j, V_j stay in shared memory and
+//      the CTA walks the single contiguous range of query tiles that see tile j (sink and
+//      interval keys are seen by every later query, band keys by the next L queries) for
+//      every query head of the group.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the
+//      elementwise softmax writes P^T and dS^T back into TMEM as bf16, where they are the A
+//      operand of dV += P^T dO and dK += dS^T Q (tcgen05 MMA with A in TMEM);
+//   3. dQ: one CTA per (b, query head h, 128-row tile i) over the forward tile plan; S and
+//      dP in TMEM, dS back into TMEM as bf16, dQ += dS K with A in TMEM.
+// Warp roles in both attention kernels: warps 0-7 elementwise softmax (two warps per TMEM
+// lane quadrant, each owning half of the columns), warp 8 TMA producer, warp 9 MMA issuer.
+#include <cuda_bf16.h>
+#include <math.h>
+
 #include "cowa_internal.h"
+#include "kernel_common.cuh"
+#include "sm100_ptx.cuh"
+
 namespace cowa {
-size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d) { return (size_t)B * Hq * N * 4; }
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t s) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kComputeWarps = 8;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kStatBytes = 1024;  // lse2[128] + delta[128] of one query tile
+
+template <int D>
+struct BwdGeom {
+  static constexpr int kTileBytes = kTile * D * 2;  // one 128-row bf16 tile of width D
+  // dK/dV kernel: K, V resident + 2 slots of {Q, dO, stats}
+  static constexpr int kSlotKV = 2 * kTileBytes + kStatBytes;
+  static constexpr int kSmemKV = 2 * kTileBytes + 2 * kSlotKV + 1024;
+  // dQ kernel: Q, dO resident + 2 slots of {K, V}
+  static constexpr int kSlotQ = 2 * kTileBytes;
+  static constexpr int kSmemQ = 2 * kTileBytes + 2 * kSlotQ + 1024;
+  static constexpr int kColAcc = 256;  // first accumulator column
+};
+
+// ------------------------------------------------------------------------------ preprocess
+// One block of 256 threads per (128-row tile, head, batch).  D/8 lanes per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_constant__ BwdArgs a) {
+  constexpr int LPR = D / 8;            // lanes per row
+  constexpr int RPI = 256 / LPR;        // rows per iteration of the block
+  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int sub = threadIdx.x % LPR, rr = threadIdx.x / LPR;
+  const size_t base = ((size_t)b * a.Hq + h) * a.N_pad;
+  for (int r = rr; r < kTile; r += RPI) {
+    const int t = i * kTile + r;
+    float acc = 0.f;
+    if (t < a.N) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + b * a.o_sb +
+                                                      (int64_t)t * a.o_st + h * a.o_sh + sub * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dO) + b * a.do_sb +
+                                                      (int64_t)t * a.do_st + h * a.do_sh + sub * 8);
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(dw[e] << 16), acc);
+        acc = fmaf(__uint_as_float(ow[e] & 0xffff0000u), __uint_as_float(dw[e] & 0xffff0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (sub == 0) {
+      a.delta[base + t] = acc;
+      a.lse2[base + t] = t < a.N ? a.lse[((size_t)b * a.Hq + h) * a.N + t] * 1.4426950408889634f : INFINITY;
+    }
+  }
 }
+
+// Pack 64 fp32 values (as two 32-column halves) into 32 bf16x2 words.
+__device__ __forceinline__ void pack64(const float* v, uint32_t* w) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = ptx::pack_bf16(v[2 * c], v[2 * c + 1]);
+}
+
+// ------------------------------------------------------------------------------ dK / dV
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+  using Geo = BwdGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full, ld_done, p_ready, acc_full,
+      mma_final;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = a.Hq / a.Hkv;
+  // lowest key tiles first: their query ranges (sink, early intervals) are the longest
+  const int j = blockIdx.x / (a.Hkv * a.B);
+  const int rem = blockIdx.x % (a.Hkv * a.B);
+  const int g = rem % a.Hkv, b = rem / a.Hkv;
+  const int s0 = j * kTile, s1 = imin(a.N, s0 + kTile);
+  const Range iv = interval_of(a.pat, g);
+  const Range rows = bwd_row_range(a.pat, iv, s0, s1, a.N);
+  const int i_lo = rows.lo / kTile, i_hi = (rows.hi + kTile - 1) / kTile;
+  const int nsteps = (i_hi - i_lo) * grp;
+
+  uint8_t* sK = smem;
+  uint8_t* sV = smem + Geo::kTileBytes;
+  uint8_t* sSlot = smem + 2 * Geo::kTileBytes;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&kv_full, 1);
+    for (int s = 0; s < 2; ++s) { ptx::mbar_init(&slot_full[s], 1); ptx::mbar_init(&slot_empty[s], 1); }
+    ptx::mbar_init(&sdp_full, 1);
+    ptx::mbar_init(&ld_done, kComputeWarps);
+    ptx::mbar_init(&p_ready, kComputeWarps);
+    ptx::mbar_init(&acc_full, 1);
+    ptx::mbar_init(&mma_final, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(&tmem_base_sh, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&a.tm_q);
+      ptx::tma_prefetch_desc(&a.tm_do);
+      ptx::mbar_arrive_expect_tx(&kv_full, 2 * Geo::kTileBytes);
+      for (int u = 0; u < D / 64; ++u) {
+        ptx::tma_load_4d(sK + u * 16384, &a.tm_k, &kv_full, u * 64, s0, g, b);
+        ptx::tma_load_4d(sV + u * 16384, &a.tm_v, &kv_full, u * 64, s0, g, b);
+      }
+      int issued = 0;
+      for (int n = 0; n < nsteps; ++n) {
+        const int slot = n & 1;
+        if (n >= 2 && !ptx::mbar_wait(&slot_empty[slot], ((n >> 1) - 1) & 1, &abort_flag, a.status)) break;
+        const int i = i_lo + n / grp, h = g * grp + n % grp;
+        uint8_t* dst = sSlot + slot * Geo::kSlotKV;
+        ptx::mbar_arrive_expect_tx(&slot_full[slot], Geo::kSlotKV);
+        for (int u = 0; u < D / 64; ++u) {
+          ptx::tma_load_4d(dst + u * 16384, &a.tm_q, &slot_full[slot], u * 64, i * kTile, h, b);
+          ptx::tma_load_4d(dst + Geo::kTileBytes + u * 16384, &a.tm_do, &slot_full[slot], u * 64, i * kTile, h, b);
+        }
+        const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + (size_t)i * kTile;
+        ptx::bulk_load(dst + 2 * Geo::kTileBytes, a.lse2 + so, 512, &slot_full[slot]);
+        ptx::bulk_load(dst + 2 * Geo::kTileBytes + 512, a.delta + so, 512, &slot_full[slot]);
+        issued = n + 1;
+      }
+      ptx::mbar_wait(&kv_full, 0, nullptr, a.status);
+      for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
+        ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, nullptr, a.status);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+      const uint32_t k_addr = ptx::smem_u32(sK), v_addr = ptx::smem_u32(sV), slot_addr = ptx::smem_u32(sSlot);
+      bool ok = ptx::mbar_wait(&kv_full, 0, &abort_flag, a.status);
+      ptx::tc_fence_after();
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const int slot = n & 1;
+        const uint32_t qa = slot_addr + slot * Geo::kSlotKV, da = qa + Geo::kTileBytes;
+        if (!(ok = ptx::mbar_wait(&slot_full[slot], (n >> 1) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + 0, ptx::smem_desc_sw128(k_addr + off, 16, 1024),
+                           ptx::smem_desc_sw128(qa + off, 16, 1024), idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + 128, ptx::smem_desc_sw128(v_addr + off, 16, 1024),
+                           ptx::smem_desc_sw128(da + off, 16, 1024), idesc_s, kk > 0);
+        }
+        ptx::mma_commit(&sdp_full);
+        if (!(ok = ptx::mbar_wait(&p_ready, n & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + 0 + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
+                           idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, tmem + 128 + kk * 8,
+                           ptx::smem_desc_sw128(qa + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(&slot_empty[slot]);
+      }
+      if (ok) ptx::mma_commit(&acc_full);
+      ptx::mma_commit(&mma_final);
+      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    }
+  } else {
+    // ------------------------------------------------------------ elementwise softmax (8 warps)
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;  // key row of the tile = TMEM lane
+    const int s = s0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const bool special = s < a.pat.S || (s >= iv.lo && s < iv.hi);
+    const int t_hi = special ? a.N : imin(a.N, s + a.pat.L);  // rows [s, t_hi) see key s
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < nsteps; ++n) {
+      const int i = i_lo + n / grp;
+      const int t0 = i * kTile;
+      const bool need_mask = !tile_full(a.pat, iv, t0, imin(a.N, t0 + kTile), s0, s1);
+      if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      uint32_t sv[64], pv[64];
+      ptx::tmem_ld32(lane_base + half * 64, sv);
+      ptx::tmem_ld32(lane_base + half * 64 + 32, sv + 32);
+      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);
+      ptx::tmem_ld32(lane_base + 128 + half * 64 + 32, pv + 32);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ld_done);
+      const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes);
+      float pf[64], df[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int col = half * 64 + c;
+        const int t = t0 + col;
+        float p = ptx::ex2(__uint_as_float(sv[c]) * sl2 - stat[col]);
+        if (need_mask && !(t >= s && t < t_hi)) p = 0.f;
+        pf[c] = p;
+        df[c] = p * (__uint_as_float(pv[c]) - stat[128 + col]);
+      }
+      uint32_t pw[32], dw[32];
+      pack64(pf, pw);
+      pack64(df, dw);
+      // every compute warp must have read S^T / dP^T before P^T / dS^T overwrite them
+      if (!(ok = ptx::mbar_wait_warp(&ld_done, n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      ptx::tmem_st32(lane_base + half * 32, pw);
+      ptx::tmem_st32(lane_base + 128 + half * 32, dw);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&p_ready);
+    }
+    if (ok && nsteps > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
+      ptx::tc_fence_after();
+      constexpr int HC = D / 2;  // accumulator columns per half
+      uint32_t dvv[HC], dkv[HC];
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) {
+        ptx::tmem_ld32(lane_base + Geo::kColAcc + half * HC + c * 32, dvv + c * 32);
+        ptx::tmem_ld32(lane_base + Geo::kColAcc + D + half * HC + c * 32, dkv + c * 32);
+      }
+      ptx::tmem_wait_ld();
+      if (s < a.N) {
+        __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + (int64_t)s * a.dv_st +
+                             g * a.dv_sh + half * HC;
+        __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + (int64_t)s * a.dk_st +
+                             g * a.dk_sh + half * HC;
+#pragma unroll
+        for (int c8 = 0; c8 < HC / 8; ++c8) {
+          uint32_t w[4], x[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[e] = ptx::pack_bf16(__uint_as_float(dvv[c8 * 8 + 2 * e]), __uint_as_float(dvv[c8 * 8 + 2 * e + 1]));
+            x[e] = ptx::pack_bf16(__uint_as_float(dkv[c8 * 8 + 2 * e]) * a.scale,
+                                  __uint_as_float(dkv[c8 * 8 + 2 * e + 1]) * a.scale);
+          }
+          reinterpret_cast<uint4*>(dvr)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
+          reinterpret_cast<uint4*>(dkr)[c8] = make_uint4(x[0], x[1], x[2], x[3]);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ dQ
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+  using Geo = BwdGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], sdp_full, ld_done, p_ready, acc_full, mma_final;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = a.Hq / a.Hkv;
+  const int nq = (a.N + kTile - 1) / kTile;
+  const int per_i = a.B * a.Hq;
+  const int i = nq - 1 - (int)(blockIdx.x / per_i);  // heaviest (last) query tiles first
+  const int rem = blockIdx.x % per_i;
+  const int h = rem % a.Hq, b = rem / a.Hq;
+  const int g = h / grp;
+  const int t0 = i * kTile, t1 = imin(a.N, t0 + kTile);
+  const Range iv = interval_of(a.pat, g);
+  const Tiles T = plan_tiles(a.pat, iv, t0, t1);
+  const int ntiles = T.count;
+
+  uint8_t* sQ = smem;
+  uint8_t* sDO = smem + Geo::kTileBytes;
+  uint8_t* sSlot = smem + 2 * Geo::kTileBytes;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&q_full, 1);
+    for (int s = 0; s < 2; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
+    ptx::mbar_init(&sdp_full, 1);
+    ptx::mbar_init(&ld_done, kComputeWarps);
+    ptx::mbar_init(&p_ready, kComputeWarps);
+    ptx::mbar_init(&acc_full, 1);
+    ptx::mbar_init(&mma_final, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(&tmem_base_sh, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      ptx::tma_prefetch_desc(&a.tm_k);
+      ptx::tma_prefetch_desc(&a.tm_v);
+      ptx::mbar_arrive_expect_tx(&q_full, 2 * Geo::kTileBytes);
+      for (int u = 0; u < D / 64; ++u) {
+        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, t0, h, b);
+        ptx::tma_load_4d(sDO + u * 16384, &a.tm_do, &q_full, u * 64, t0, h, b);
+      }
+      TileCursor cur;
+      cur.init(T);
+      int issued = 0;
+      for (int n = 0; n < ntiles; ++n, cur.next(T)) {
+        const int slot = n & 1;
+        if (n >= 2 && !ptx::mbar_wait(&kv_empty[slot], ((n >> 1) - 1) & 1, &abort_flag, a.status)) break;
+        uint8_t* dst = sSlot + slot * Geo::kSlotQ;
+        ptx::mbar_arrive_expect_tx(&kv_full[slot], Geo::kSlotQ);
+        for (int u = 0; u < D / 64; ++u) {
+          ptx::tma_load_4d(dst + u * 16384, &a.tm_k, &kv_full[slot], u * 64, cur.j * kTile, g, b);
+          ptx::tma_load_4d(dst + Geo::kTileBytes + u * 16384, &a.tm_v, &kv_full[slot], u * 64, cur.j * kTile, g, b);
+        }
+        issued = n + 1;
+      }
+      ptx::mbar_wait(&q_full, 0, nullptr, a.status);
+      for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
+        ptx::mbar_wait(&kv_full[n & 1], (n >> 1) & 1, nullptr, a.status);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+      const uint32_t q_addr = ptx::smem_u32(sQ), do_addr = ptx::smem_u32(sDO), slot_addr = ptx::smem_u32(sSlot);
+      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
+      ptx::tc_fence_after();
+      for (int n = 0; ok && n < ntiles; ++n) {
+        const int slot = n & 1;
+        const uint32_t ka = slot_addr + slot * Geo::kSlotQ, va = ka + Geo::kTileBytes;
+        if (!(ok = ptx::mbar_wait(&kv_full[slot], (n >> 1) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + 0, ptx::smem_desc_sw128(q_addr + off, 16, 1024),
+                           ptx::smem_desc_sw128(ka + off, 16, 1024), idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          ptx::mma_bf16_ss(tmem + 128, ptx::smem_desc_sw128(do_addr + off, 16, 1024),
+                           ptx::smem_desc_sw128(va + off, 16, 1024), idesc_s, kk > 0);
+        }
+        ptx::mma_commit(&sdp_full);
+        if (!(ok = ptx::mbar_wait(&p_ready, n & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        // dQ += dS K : A = dS in TMEM, B = K MN-major in smem
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + 0 + kk * 8, ptx::smem_desc_sw128(ka + kk * 2048, 16384, 1024),
+                           idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(&kv_empty[slot]);
+      }
+      if (ok) ptx::mma_commit(&acc_full);
+      ptx::mma_commit(&mma_final);
+      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    }
+  } else {
+    const int quad = warp & 3, half = warp >> 2;
+    const int r = quad * 32 + lane;  // query row = TMEM lane
+    const int t = t0 + r;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + t;
+    const float lse2 = a.lse2[so], delta = a.delta[so];
+    const float sl2 = a.scale_log2;
+    // visible key ranges of row t (absolute positions)
+    const int sink_end = imin(a.pat.S, t + 1);
+    const int band_lo = imax(0, t - a.pat.L + 1);
+    const int lr_lo = iv.lo, lr_hi = imin(iv.hi, t + 1);
+    bool ok = true;
+    TileCursor cur;
+    cur.init(T);
+    for (int n = 0; n < ntiles; ++n, cur.next(T)) {
+      const int s0 = cur.j * kTile;
+      const bool need_mask = (s0 + kTile > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kTile));
+      if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      uint32_t sv[64], pv[64];
+      ptx::tmem_ld32(lane_base + half * 64, sv);
+      ptx::tmem_ld32(lane_base + half * 64 + 32, sv + 32);
+      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);
+      ptx::tmem_ld32(lane_base + 128 + half * 64 + 32, pv + 32);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&ld_done);
+      float df[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int s = s0 + half * 64 + c;
+        float p = ptx::ex2(__uint_as_float(sv[c]) * sl2 - lse2);
+        if (need_mask) {
+          const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
+          if (!vis) p = 0.f;
+        }
+        df[c] = p * (__uint_as_float(pv[c]) - delta);
+      }
+      uint32_t dw[32];
+      pack64(df, dw);
+      if (!(ok = ptx::mbar_wait_warp(&ld_done, n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      ptx::tmem_st32(lane_base + half * 32, dw);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&p_ready);
+    }
+    if (ok && ntiles > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
+      ptx::tc_fence_after();
+      constexpr int HC = D / 2;
+      uint32_t dqv[HC];
+#pragma unroll
+      for (int c = 0; c < HC / 32; ++c) ptx::tmem_ld32(lane_base + Geo::kColAcc + half * HC + c * 32, dqv + c * 32);
+      ptx::tmem_wait_ld();
+      if (t < a.N) {
+        __nv_bfloat16* dqr = reinterpret_cast<__nv_bfloat16*>(a.dq) + b * a.dq_sb + (int64_t)t * a.dq_st +
+                             h * a.dq_sh + half * HC;
+#pragma unroll
+        for (int c8 = 0; c8 < HC / 8; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = ptx::pack_bf16(__uint_as_float(dqv[c8 * 8 + 2 * e]) * a.scale,
+                                  __uint_as_float(dqv[c8 * 8 + 2 * e + 1]) * a.scale);
+          reinterpret_cast<uint4*>(dqr)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
+  using Geo = BwdGeom<D>;
+  const int nq = a.N_pad / kTile;
+  bwd_preprocess_kernel<D><<<dim3(nq, a.Hq, a.B), 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kdkdv = bwd_dkdv_kernel<D>;
+  auto kdq = bwd_dq_kernel<D>;
+  if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemKV)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemQ)) != cudaSuccess)
+    return e;
+  const long long n_kv = (long long)nq * a.Hkv * a.B;
+  const long long n_q = (long long)nq * a.Hq * a.B;
+  if (n_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+  kdkdv<<<(unsigned)n_kv, kThreads, Geo::kSmemKV, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kdq<<<(unsigned)n_q, kThreads, Geo::kSmemQ, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d) {
+  (void)Hkv; (void)d;
+  const size_t n_pad = (size_t)(N + kTile - 1) / kTile * kTile;
+  return align_up(2 * (size_t)B * Hq * n_pad * sizeof(float), 256);
+}
+
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t s) {
+  if (a.d == 64) return launch_bwd_d<64>(a, s);
+  if (a.d == 128) return launch_bwd_d<128>(a, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cowa

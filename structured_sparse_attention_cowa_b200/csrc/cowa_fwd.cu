@@ -20,12 +20,13 @@
 #include <math.h>
 
 #include "cowa_internal.h"
+#include "kernel_common.cuh"
 #include "sm100_ptx.cuh"
 
 namespace cowa {
 namespace {
 
-constexpr int kBM = 128, kBN = 128;
+constexpr int kBM = kTile, kBN = kTile;
 constexpr int kFwdThreads = 320;
 constexpr int kRing = 3;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
@@ -41,29 +42,6 @@ struct FwdGeom {
   static constexpr int kOffP = kOffRing + kRing * kKVBytes;
   static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;  // + alignment slack
   static constexpr int kColO = 256;
-};
-
-struct Tiles {
-  Range r[3];
-  int n;     // number of ranges
-  int count; // number of tiles
-};
-
-__device__ __forceinline__ Tiles plan_tiles(const Pat& p, Range iv, int t0, int t1) {
-  Tiles T;
-  T.n = fwd_tile_ranges(p, iv, t0, t1, kBN, T.r);
-  T.count = 0;
-  for (int x = 0; x < T.n; ++x) T.count += T.r[x].hi - T.r[x].lo;
-  return T;
-}
-
-// Walks the tile list in order.
-struct TileCursor {
-  int x, j;
-  __device__ __forceinline__ void init(const Tiles& T) { x = 0; j = T.n > 0 ? T.r[0].lo : 0; }
-  __device__ __forceinline__ void next(const Tiles& T) {
-    if (++j >= T.r[x].hi && x + 1 < T.n) { ++x; j = T.r[x].lo; }
-  }
 };
 
 template <int D>

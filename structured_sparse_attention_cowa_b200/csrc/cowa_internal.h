@@ -64,7 +64,9 @@ struct BwdArgs {
   void* dq; int64_t dq_sb, dq_st, dq_sh;
   void* dk; int64_t dk_sb, dk_st, dk_sh;
   void* dv; int64_t dv_sb, dv_st, dv_sh;
-  float* delta;      // [B, Hq, N] fp32 workspace
+  float* delta;      // [B, Hq, N_pad] fp32 workspace: rowsum(dO * O), 0 on padded rows
+  float* lse2;       // [B, Hq, N_pad] fp32 workspace: lse * log2(e), +inf on padded rows
+  int N_pad;         // N rounded up to a whole number of 128-row tiles
   uint32_t* status;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)

@@ -1,0 +1,114 @@
+"""GPU parity: cowa_bwd (through the C ABI) against the fp64 oracle.
+
+Tolerance: relative Frobenius error <= 1e-2 for dq, dk, dv against fp64 gradients of
+sum(dO * O) on identical bf16 inputs.  The forward output o and lse fed to the backward
+come from cowa_fwd (as in training); the oracle recomputes everything from q, k, v, dO."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import cowa_oracle as orc
+from structured_sparse_attention_cowa_b200 import cowa as cw
+from structured_sparse_attention_cowa_b200 import synth
+from tests.gpu_helpers import GRAD_RTOL, DeviceView, edge_rows, host_and_device, oracle_pattern, rel_fro, to64
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(B, N, Hq, Hkv, d, device, extra=0, cuda_gen=False):
+    if cuda_gen:
+        t = [synth.cuda_normal_bf16(s, synth.seed_of(n, extra), device)
+             for s, n in (((B, N, Hq, d), "q"), ((B, N, Hkv, d), "k"), ((B, N, Hkv, d), "v"), ((B, N, Hq, d), "do"))]
+        return [DeviceView(x) for x in t], t
+    pairs = [host_and_device(s, n, device, extra)
+             for s, n in (((B, N, Hq, d), "q"), ((B, N, Hkv, d), "k"), ((B, N, Hkv, d), "v"), ((B, N, Hq, d), "do"))]
+    return [p[0] for p in pairs], [p[1] for p in pairs]
+
+
+def _run(dev_inputs, pat):
+    q, k, v, do = dev_inputs
+    o, lse = cw.cowa_fwd(q, k, v, pat)
+    dq, dk, dv = cw.cowa_bwd(q, k, v, o, lse, do, pat)
+    torch.cuda.synchronize()
+    return dq, dk, dv
+
+
+def _check_full(B, N, Hq, Hkv, d, pat, device, extra=0):
+    host, dev = _inputs(B, N, Hq, Hkv, d, device, extra)
+    dq, dk, dv = _run(dev, pat)
+    wq, wk, wv = orc.attention_bwd(*host, oracle_pattern(pat))
+    errs = (rel_fro(to64(dq), wq), rel_fro(to64(dk), wk), rel_fro(to64(dv), wv))
+    assert max(errs) <= GRAD_RTOL, errs
+
+
+@pytest.mark.parametrize("D", [4, 2, 1])
+def test_bwd_tiny_config(cuda_device, D):
+    """B=1, N=T=1024, H_q=8, H_kv=4, d=64, S=64, L=128; D=4 and the duplicated D=2, 1."""
+    _check_full(1, 1024, 8, 4, 64, cw.Pattern(64, 128, 1024, D), cuda_device)
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,pat", [
+    (1, 1000, 10, 2, 128, cw.Pattern(64, 128, 1000, 2)),     # ragged tail, group of 5
+    (2, 333, 4, 4, 128, cw.Pattern(5, 40, 333, 4)),          # group of 1, unaligned sink
+    (1, 77, 6, 2, 64, cw.Pattern(0, 1, 77, 2)),              # one partial tile, L = 1
+    (1, 640, 8, 2, 128, cw.Pattern(16, 640, 640, 2)),        # dense causal
+    (1, 520, 4, 2, 64, cw.Pattern(4, 60, 4, 1)),             # SWA + sinks
+    (1, 700, 8, 4, 128, cw.Pattern(32, 100, 500, 4)),        # N > T
+    (1, 300, 2, 1, 128, cw.Pattern(7, 30, 300, 2, kv_head_base=1, h_kv_global=2)),  # TP rank
+    (1, 256, 16, 2, 64, cw.Pattern(16, 64, 256, 2, softmax_scale=0.3)),  # group of 8
+])
+def test_bwd_edge_shapes(cuda_device, B, N, Hq, Hkv, d, pat):
+    _check_full(B, N, Hq, Hkv, d, pat, cuda_device, extra=2)
+
+
+def _check_sampled(B, N, Hq, Hkv, d, pat, device, rows, col_sets, cuda_gen):
+    """dq on sampled rows (all heads) and dk/dv on sampled columns of some KV heads."""
+    host, dev = _inputs(B, N, Hq, Hkv, d, device, cuda_gen=cuda_gen)
+    dq, dk, dv = _run(dev, pat)
+    op = oracle_pattern(pat)
+    rows_t = torch.as_tensor(rows, device=device)
+    wq = orc.attention_bwd_rows(*host, op, rows, b=0)
+    assert rel_fro(to64(dq[0, rows_t]), wq) <= GRAD_RTOL
+    for g, cols in col_sets:
+        wk, wv = orc.attention_bwd_cols(*host, op, b=0, g=g, cols=cols)
+        ct = torch.as_tensor(cols, device=device)
+        assert rel_fro(to64(dk[0, ct, g]), wk) <= GRAD_RTOL, ("dk", g)
+        assert rel_fro(to64(dv[0, ct, g]), wv) <= GRAD_RTOL, ("dv", g)
+    # properties that hold at any size: softmax rows sum to one, and a shift of every key
+    # by the same vector leaves the output unchanged
+    grp = Hq // Hkv
+    sum_dv = dv.double().sum(1)            # [B, Hkv, d]
+    sum_do = dev[3].double().sum(1).view(B, Hkv, grp, d).sum(2)
+    assert float((sum_dv - sum_do).norm() / sum_do.norm()) <= GRAD_RTOL
+    sum_dk = dk.double().sum(1)
+    assert float(sum_dk.norm() / dk.double().norm()) <= GRAD_RTOL
+    return dq, dk, dv
+
+
+def test_bwd_prefill_8k(cuda_device):
+    """B=2, N=T=8192, H_q=32, H_kv=8, d=128, S=128, L=1024, D=8."""
+    pat = cw.Pattern(128, 1024, 8192, 8)
+    rows = edge_rows(8192, pat, 8, extra_random=128, seed=5)
+    cols = [0, 127, 128, 129, 1100, 1151, 5000, 8191]
+    _check_sampled(2, 8192, 32, 8, 128, pat, cuda_device, rows, [(0, cols), (7, cols)], cuda_gen=False)
+
+
+def test_bwd_train_32k(cuda_device):
+    """B=1, N=T=32768, H_q=40, H_kv=8, d=128, S=128, L=2048, D=8: sampled rows, band-only and
+    late-interval columns, and the any-size identities."""
+    pat = cw.Pattern(128, 2048, 32768, 8)
+    rows = edge_rows(32768, pat, 8, extra_random=96, seed=6)
+    band_cols = [5000, 5001, 9000, 20000]
+    late = [28688, 28700, 30000, 32767]   # interval of KV head 7 and the last key
+    _check_sampled(1, 32768, 40, 8, 128, pat, cuda_device, rows, [(0, band_cols), (7, band_cols + late)],
+                   cuda_gen=True)
+
+
+def test_bwd_long_128k(cuda_device):
+    """B=1, N=T=131072, H_q=40, H_kv=8, d=128, S=128, L=4096, D=8: sampled rows, band-only
+    columns and the any-size identities."""
+    pat = cw.Pattern(128, 4096, 131072, 8)
+    rows = np.array([0, 127, 128, 4095, 4096, 16495, 16496, 70000, 131071])
+    _check_sampled(1, 131072, 40, 8, 128, pat, cuda_device, rows, [(3, [20000, 50001]), (7, [131071])],
+                   cuda_gen=True)

@@ -319,6 +319,8 @@ def test_row_and_column_restricted_evaluation():
     np.testing.assert_allclose(orow, o[0, rows], atol=1e-12)
     np.testing.assert_allclose(lrow, lse[0][:, rows].T, atol=1e-12)
     dq, dk, dv = orc.attention_bwd(q, k, v, do, pat)
+    dqr = orc.attention_bwd_rows(q, k, v, do, pat, rows, b=0)
+    np.testing.assert_allclose(dqr, dq[0, rows], atol=1e-10)
     cols = [0, 4, 6, 30, 44, 79]
     for g in range(Hkv):
         dkc, dvc = orc.attention_bwd_cols(q, k, v, do, pat, b=0, g=g, cols=cols, row_block=17)
