@@ -113,6 +113,28 @@ def _traffic_record(kernel_file: str):
     return None
 
 
+# ------------------------------------------------------------------------------ multi-rank
+def rank_seed_extra(rank: int) -> int:
+    """Each rank draws its own batch element (weak scaling by batch sharding)."""
+    return rank
+
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, flop_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: all ranks' work over the max-over-ranks step time."""
+    return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
@@ -130,7 +152,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -238,7 +260,7 @@ def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cowa", choices=["cowa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -297,7 +319,7 @@ def run_cowa(args, world, rank, local):
     dpat = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
 
     # ---- inputs (per rank: its own batch element / seeds), outputs, workspaces
-    ex = rank
+    ex = rank_seed_extra(rank)
     q = synth.cuda_normal_bf16((c["B"], c["N"], c["Hq"], c["d"]), synth.seed_of("q", ex), dev)
     k = synth.cuda_normal_bf16((c["B"], c["N"], c["Hkv"], c["d"]), synth.seed_of("k", ex), dev)
     v = synth.cuda_normal_bf16((c["B"], c["N"], c["Hkv"], c["d"]), synth.seed_of("v", ex), dev)
@@ -337,11 +359,7 @@ def run_cowa(args, world, rank, local):
             dist.barrier()
 
     def maxr(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(x, dist, dev)
 
     # ---- warm-up
     for _ in range(max(3, args.warmup)):
@@ -375,7 +393,7 @@ def run_cowa(args, world, rank, local):
     toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
     dec_bytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2  # K and V rows, bf16
     ms_step = total_ms / K
-    value = world * (fwd_flop + bwd_flop) / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(world, fwd_flop + bwd_flop, ms_step)
 
     burst, sustained, hbm, peak_src = _peaks()
     parts = {
@@ -439,7 +457,7 @@ def run_cowa(args, world, rank, local):
         b.record(); torch.cuda.synchronize()
         barrier()
         e_ms = maxr(a.elapsed_time(b)) / KE
-        e2e = {"value": world * (fwd_flop + bwd_flop) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE}
 
     cpu = None
