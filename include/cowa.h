@@ -122,6 +122,32 @@ cowa_status cowa_decode(const cowa_pattern* pat, int B, int H_q, int H_kv, int d
                         const int32_t* pos, void* o, float* lse_or_null,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* ---- decode without a caller workspace -----------------------------------------------------
+ * This entry point has no counterpart on the CoWA pages; it is a convenience of this library for
+ * callers that cannot allocate device memory (runtimes that reserve the whole memory pool up
+ * front and forbid allocations on the serving path, or code that must not call cudaMalloc
+ * because it would synchronize the device).
+ *
+ * Same inputs, outputs and result as cowa_decode, but no workspace argument: the split partials
+ * and the status word live in a scratch array of COWA_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) that is
+ * a static device variable of the library.  Every GPU that loads the library holds one copy of it
+ * until the process exits.  The call allocates nothing (no cudaMalloc, no allocating library
+ * routine).
+ *   - The first call made with a given device current looks up the scratch address on that
+ *     device (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call shares the one scratch array of its device and leaves its contents behind.
+ *     The status word is cleared at the start of each call.  Calls that overlap on the GPU
+ *     (e.g. on two streams without ordering between them) race on the scratch and give
+ *     undefined results: order them on one stream or synchronize between them.
+ *   - A configuration whose workspace (cowa_decode_workspace_size) exceeds the scratch size
+ *     returns COWA_ERR_WORKSPACE without launching.  Other argument errors are those of
+ *     cowa_decode.  A device-side timeout leaves its status in the library's scratch, which the
+ *     caller cannot read: use cowa_decode when the status matters. */
+#define COWA_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+cowa_status cowa_decode_noalloc(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap,
+                                const void* q_t, cowa_tensor k_cache, cowa_tensor v_cache,
+                                const int32_t* pos, void* o, float* lse_or_null, void* stream);
+
 /* ---- status --------------------------------------------------------------------------------
  * Synchronizes `stream`, reads and clears the device status word in `ws` (the workspace of an
  * earlier call), and returns COWA_OK or COWA_ERR_TIMEOUT (COWA_ERR_CUDA if the stream failed). */

@@ -27,7 +27,7 @@ _STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED", 3
 
 EXPORTED = ["cowa_fwd_workspace_size", "cowa_fwd", "cowa_bwd_workspace_size", "cowa_bwd",
             "cowa_decode_workspace_size", "cowa_decode", "cowa_workspace_status", "cowa_status_string",
-            "cowa_visible_counts", "cowa_plan_debug", "cowa_version"]
+            "cowa_visible_counts", "cowa_plan_debug", "cowa_version", "cowa_decode_noalloc"]
 
 
 class CowaError(RuntimeError):
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.cowa_decode_workspace_size.restype = sz
     L.cowa_decode.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp, sz, vp]
     L.cowa_decode.restype = i
+    L.cowa_decode_noalloc.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp]
+    L.cowa_decode_noalloc.restype = i
     L.cowa_workspace_status.argtypes = [vp, vp]
     L.cowa_workspace_status.restype = i
     L.cowa_status_string.argtypes = [i]
@@ -216,6 +218,26 @@ def cowa_decode(q_t, k_cache, v_cache, pos, pattern: Pattern, layout: str = "bht
                                         _cache_tensor(k_cache, layout), _cache_tensor(v_cache, layout),
                                         pos.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
                                         workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def cowa_decode_noalloc(q_t, k_cache, v_cache, pos, pattern: Pattern, out, lse=None, layout: str = "bhtd",
+                        stream=None):
+    """cowa_decode without a workspace: the library's static per-device scratch holds the split
+    partials (see include/cowa.h).  `out` [B,H_q,d] bf16 (and `lse` [B,H_q] fp32, optional) are
+    the caller's; nothing is allocated by this call."""
+    for n_, x_ in (("q_t", q_t), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+        _bf16_cuda(n_, x_)
+    B, Hq, d = q_t.shape
+    if layout == "bhtd":
+        Hkv, T_cap = k_cache.shape[1], k_cache.shape[2]
+    else:
+        T_cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    pat = pattern.c()
+    _check("cowa_decode_noalloc", lib().cowa_decode_noalloc(
+        ctypes.byref(pat), B, Hq, Hkv, d, T_cap, q_t.data_ptr(), _cache_tensor(k_cache, layout),
+        _cache_tensor(v_cache, layout), pos.data_ptr(), out.data_ptr(),
+        lse.data_ptr() if lse is not None else None, _stream(stream)))
     return out, lse
 
 
