@@ -5,14 +5,17 @@
 //
 // HBM-bound: per (b, g) only the <= 3 visible token ranges at pos[b] (sink, interval_g,
 // near-diagonal band) are read.  Each CTA owns one chunk of one range:
-//   * a producer warp streams 64-token K and V sub-tiles into a shared-memory ring with
-//     TMA (128-byte swizzle, coalesced 128-byte rows, no register staging);
-//   * 8 compute warps: 8 lanes per token row, each lane one 16-byte unit per 64-wide
-//     slice of d (128-bit shared loads, conflict-free under the swizzle), scores for all
-//     query heads of the GQA group from fp32 registers, a 3-step shuffle reduction, an
-//     online softmax in the log2 domain, and P*V accumulation in fp32;
-//   * the lanes' partial (m, l, o) states are merged with shuffles, then across warps in
-//     shared memory, and written as one fp32 partial per (b, h, split).
+//   * a producer warp streams 64-token K and V sub-tiles into a shared-memory ring with TMA
+//     (128-byte swizzle, whole 128-byte rows, nothing staged through registers);
+//   * 4 compute warps each take 16 tokens of every sub-tile.  Per (b, g) decode is the
+//     contraction [grp x d] . [d x n]: scores and P.V run on warp-level tensor-core MMAs
+//     (m16n8k16, bf16 in, fp32 accumulate; the grp query heads are rows 0..grp-1 of the 16-row
+//     A operand), with K fragments from ldmatrix and V fragments from ldmatrix.trans on the
+//     swizzled tiles.  This keeps the instruction count per token small enough that the
+//     kernel is limited by HBM, not by the CUDA cores;
+//   * online softmax in the log2 domain with a lazy rescale of the accumulators;
+//   * the warps' partial (m, l, o) states are merged in shared memory and written as one fp32
+//     partial per (b, h, split).
 // A second kernel merges the splits of each (b, h) (max / rescaled sums, warp shuffles)
 // and writes bf16 o and the fp32 lse.
 #include <cuda_bf16.h>
@@ -24,28 +27,24 @@
 namespace cowa {
 namespace {
 
-constexpr int kDecWarps = 8;                        // compute warps per CTA
+constexpr int kDecWarps = 4;                        // compute warps per CTA
 constexpr int kDecThreads = (kDecWarps + 1) * 32;   // + one TMA producer warp
 constexpr int kSubTok = 64;                         // tokens per sub-tile (TMA box rows)
 constexpr int kStages = 3;                          // sub-tile ring depth
 constexpr int kBoxBytes = kSubTok * 128;            // one [64 rows x 64 bf16] box
+constexpr float kDecRescale = 8.0f;                 // lazy-rescale threshold, log2 units
 
 template <int D>
 struct DecGeom {
-  static constexpr int kUnits = D / 64;                  // 16-byte units per lane per row
-  static constexpr int kEPT = 8 * kUnits;                // elements per lane
+  static constexpr int kUnits = D / 64;                  // boxes per row
   static constexpr int kTileBytes = kUnits * kBoxBytes;  // K (or V) sub-tile
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 };
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
+// shared address of 16-byte unit u (d elements 8u..8u+7) of token row r of a swizzled tile
+__device__ __forceinline__ uint32_t unit_addr(uint32_t tile, int r, int u) {
+  return tile + (u >> 3) * kBoxBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
 }
 
 __device__ __forceinline__ float safe_ex2_diff(float a, float m) {
@@ -55,7 +54,10 @@ __device__ __forceinline__ float safe_ex2_diff(float a, float m) {
 
 template <int GRP, int D>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+  static_assert(GRP >= 1 && GRP <= 8, "query heads per KV head must fit the MMA's first 8 rows");
   using Geo = DecGeom<D>;
+  constexpr int KS = D / 16;  // k-steps of the score MMA
+  constexpr int NT = D / 8;   // n-tiles of the P.V MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -125,152 +127,120 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   }
 
   // ------------------------------------------------------------------ compute warps
-  constexpr int EPT = Geo::kEPT;
-  const int slot = lane >> 3;  // token slot of a 4-token step
-  const int j = lane & 7;      // 16-byte unit within each 64-element slice of d
-  float q[GRP][EPT];
-  float acc[GRP][EPT];
-  float m[GRP], l[GRP];
+  const int gr = lane >> 2;  // fragment row = query head of the group (rows >= GRP are zero)
+  const int tq = lane & 3;   // fragment column pair
+  // A fragments of Q (rows 8..15 of the 16-row operand are zero: a1 = a3 = 0)
+  uint32_t qa[KS][2];
   {
-    const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q_t) + ((size_t)b * a.Hq + (size_t)g * GRP) * D;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        reinterpret_cast<const __nv_bfloat16*>(a.q_t) + ((size_t)b * a.Hq + (size_t)g * GRP + imin(gr, GRP - 1)) * D);
 #pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-#pragma unroll
-      for (int u = 0; u < Geo::kUnits; ++u) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qb + hh * D + u * 64 + j * 8);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          q[hh][u * 8 + 2 * e] = bf16lo(ww[e]) * a.scale_log2;
-          q[hh][u * 8 + 2 * e + 1] = bf16hi(ww[e]) * a.scale_log2;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) acc[hh][e] = 0.f;
-      m[hh] = -INFINITY;
-      l[hh] = 0.f;
+    for (int kk = 0; kk < KS; ++kk) {
+      qa[kk][0] = gr < GRP ? qrow[8 * kk + tq] : 0u;
+      qa[kk][1] = gr < GRP ? qrow[8 * kk + 4 + tq] : 0u;
     }
   }
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float m_used = -INFINITY, lsum = 0.f;
 
   const uint32_t smem_base = ptx::smem_u32(smem);
+  const int row0 = warp * 16;  // this warp's tokens within each sub-tile
   bool ok = true;
   for (int st = 0; st < nsub; ++st) {
     const int s = st % kStages;
     if (!ptx::mbar_wait_warp(&full_bar[s], (st / kStages) & 1, &abort_flag, a.status)) { ok = false; break; }
-    const uint32_t ks = smem_base + s * Geo::kStageBytes;
-    const uint32_t vs = ks + Geo::kTileBytes;
+    const uint32_t kt = smem_base + s * Geo::kStageBytes;
+    const uint32_t vt = kt + Geo::kTileBytes;
+    // ---- scores S[head][token] for two 8-token n-tiles
+    float sc[2][4];
 #pragma unroll
-    for (int step = 0; step < kSubTok / (kDecWarps * 4); ++step) {
-      const int r = warp * (kSubTok / kDecWarps) + step * 4 + slot;  // row in the sub-tile
-      const int tok = c_lo + st * kSubTok + r;
-      const bool valid = tok < c_hi;
-      const uint32_t off = r * 128 + ((j ^ (r & 7)) << 4);  // 128-byte swizzle
-      float sc[GRP];
+    for (int nt = 0; nt < 2; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < GRP; ++hh) sc[hh] = 0.f;
-#pragma unroll
-      for (int u = 0; u < Geo::kUnits; ++u) {
-        const uint4 kw = lds128(ks + u * kBoxBytes + off);
-        const uint32_t ww[4] = {kw.x, kw.y, kw.z, kw.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float k0 = bf16lo(ww[e]), k1 = bf16hi(ww[e]);
-#pragma unroll
-          for (int hh = 0; hh < GRP; ++hh) {
-            sc[hh] = fmaf(q[hh][u * 8 + 2 * e], k0, sc[hh]);
-            sc[hh] = fmaf(q[hh][u * 8 + 2 * e + 1], k1, sc[hh]);
-          }
-        }
+      for (int k2 = 0; k2 < KS / 2; ++k2) {
+        uint32_t bb[4];
+        ptx::ldsm_x4(unit_addr(kt, row0 + 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
+        const uint32_t a0[4] = {qa[2 * k2][0], 0u, qa[2 * k2][1], 0u};
+        const uint32_t a1[4] = {qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u};
+        ptx::mma_16816(sc[nt], a0, bb[0], bb[1]);
+        ptx::mma_16816(sc[nt], a1, bb[2], bb[3]);
       }
-      float p[GRP];
+    }
+    // ---- online softmax (log2 domain) over this warp's 16 tokens
+    const int tok0 = c_lo + st * kSubTok + row0 + 2 * tq;
+    float x[4];
 #pragma unroll
-      for (int hh = 0; hh < GRP; ++hh) {
-        float x = sc[hh];
-        x += __shfl_xor_sync(0xffffffffu, x, 1);
-        x += __shfl_xor_sync(0xffffffffu, x, 2);
-        x += __shfl_xor_sync(0xffffffffu, x, 4);
-        x = valid ? x : -INFINITY;
-        if (x > m[hh]) {
-          const float f = safe_ex2_diff(m[hh], x);
-          l[hh] *= f;
+    for (int e = 0; e < 4; ++e) {
+      const int tok = tok0 + 8 * (e >> 1) + (e & 1);
+      x[e] = tok < c_hi ? sc[e >> 1][e & 1] * a.scale_log2 : -INFINITY;
+    }
+    float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_used, mx);
+    if (m_new != -INFINITY && (m_used == -INFINITY || m_new > m_used + kDecRescale)) {
+      const float alpha = ptx::ex2(m_used - m_new);  // 0 when nothing was visible before
+      lsum *= alpha;
 #pragma unroll
-          for (int e = 0; e < EPT; ++e) acc[hh][e] *= f;
-          m[hh] = x;
-        }
-        p[hh] = valid ? ptx::ex2(x - m[hh]) : 0.f;
-        l[hh] += p[hh];
-      }
+      for (int n = 0; n < NT; ++n) { acc[n][0] *= alpha; acc[n][1] *= alpha; }
+      m_used = m_new;
+    }
+    const float m_eff = m_used == -INFINITY ? 0.f : m_used;
+    float p[4];
 #pragma unroll
-      for (int u = 0; u < Geo::kUnits; ++u) {
-        const uint4 vw = lds128(vs + u * kBoxBytes + off);
-        const uint32_t ww[4] = {vw.x, vw.y, vw.z, vw.w};
+    for (int e = 0; e < 4; ++e) {
+      p[e] = ptx::ex2(x[e] - m_eff);
+      lsum += p[e];
+    }
+    // P as the A operand: tokens 2tq, 2tq+1 (first n-tile) and 8+2tq, 9+2tq (second)
+    const uint32_t pa[4] = {ptx::pack_bf16(p[0], p[1]), 0u, ptx::pack_bf16(p[2], p[3]), 0u};
+    // ---- O[head][d] += P[head][token] V[token][d]
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float v0 = bf16lo(ww[e]), v1 = bf16hi(ww[e]);
-#pragma unroll
-          for (int hh = 0; hh < GRP; ++hh) {
-            acc[hh][u * 8 + 2 * e] = fmaf(p[hh], v0, acc[hh][u * 8 + 2 * e]);
-            acc[hh][u * 8 + 2 * e + 1] = fmaf(p[hh], v1, acc[hh][u * 8 + 2 * e + 1]);
-          }
-        }
-      }
+    for (int np = 0; np < NT / 2; ++np) {
+      uint32_t bb[4];
+      ptx::ldsm_x4_trans(unit_addr(vt, row0 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
+      ptx::mma_16816(acc[2 * np], pa, bb[0], bb[1]);
+      ptx::mma_16816(acc[2 * np + 1], pa, bb[2], bb[3]);
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
   }
-
-  // ---- merge the four token slots of the warp (lanes j, j+8, j+16, j+24)
-#pragma unroll
-  for (int offs = 8; offs <= 16; offs <<= 1) {
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[hh], offs);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[hh], offs);
-      const float mn = fmaxf(m[hh], mo);
-      const float fa = safe_ex2_diff(m[hh], mn), fb = safe_ex2_diff(mo, mn);
-      l[hh] = l[hh] * fa + lo * fb;
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][e], offs);
-        acc[hh][e] = acc[hh][e] * fa + ao * fb;
-      }
-      m[hh] = mn;
-    }
-  }
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
 
   // ---- merge the warps through shared memory (the ring is drained: reuse it)
   asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32) : "memory");
   if (!ok || abort_flag) return;
-  float* red = reinterpret_cast<float*>(smem);  // [warp][GRP][D + 2]
-  if (lane < 8) {
+  float* red = reinterpret_cast<float*>(smem);  // [warp][8 rows][D + 2]
+  {
+    float* rw = red + (warp * 8 + gr) * (D + 2);
+    if (tq == 0) { rw[0] = m_used; rw[1] = lsum; }
 #pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-      float* rw = red + (warp * GRP + hh) * (D + 2);
-      if (lane == 0) { rw[0] = m[hh]; rw[1] = l[hh]; }
-#pragma unroll
-      for (int u = 0; u < Geo::kUnits; ++u)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rw[2 + u * 64 + j * 8 + e] = acc[hh][u * 8 + e];
+    for (int n = 0; n < NT; ++n) {
+      rw[2 + 8 * n + 2 * tq] = acc[n][0];
+      rw[2 + 8 * n + 2 * tq + 1] = acc[n][1];
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32) : "memory");
-  for (int x = threadIdx.x; x < GRP * D; x += kDecWarps * 32) {
-    const int hh = x / D, dc = x % D;
-    float mx = -INFINITY;
+  for (int xi = threadIdx.x; xi < GRP * D; xi += kDecWarps * 32) {
+    const int hh = xi / D, dc = xi % D;
+    float mxw = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) mx = fmaxf(mx, red[(w * GRP + hh) * (D + 2)]);
+    for (int w = 0; w < kDecWarps; ++w) mxw = fmaxf(mxw, red[(w * 8 + hh) * (D + 2)]);
     float o = 0.f, ll = 0.f;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) {
-      const float* rw = red + (w * GRP + hh) * (D + 2);
-      const float f = safe_ex2_diff(rw[0], mx);
+      const float* rw = red + (w * 8 + hh) * (D + 2);
+      const float f = safe_ex2_diff(rw[0], mxw);
       o += f * rw[2 + dc];
       ll += f * rw[1];
     }
     const int h = g * GRP + hh;
     float* out = a.partials + (((size_t)b * a.Hq + h) * a.n_split + split) * (D + 2);
     out[2 + dc] = o;
-    if (dc == 0) { out[0] = mx; out[1] = ll; }
+    if (dc == 0) { out[0] = mxw; out[1] = ll; }
   }
 }
 

@@ -4,22 +4,38 @@
 //
 // One CTA = (batch b, KV head g, 128-row query tile i, a pair of query heads of g's GQA
 // group).  The two heads share every K/V tile the CTA loads and the same tile plan, because
-// the mask depends on g only.  Warp roles (10 warps):
+// the mask depends on g only.  Warp roles (12 warps = 3 warpgroups):
 //   warps 0-3  softmax for head slot 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax for head slot 1
-//   warp  8    TMA producer: Q once, then K_j, V_j of every visited KV tile into a 3-deep ring
+//   warp  8    TMA producer: Q once, then K_j, V_j of every visited KV tile into a 4-deep ring
 //   warp  9    tcgen05 MMA issuer (one lane): S = Q K^T into TMEM, O += P V into TMEM
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: the kernel is compiled for 168 per thread (384 * 168 = 64512 at launch); the two
+// softmax warpgroups then raise theirs to 216 and the third lowers to 72
+// (2*128*216 + 128*72 = 64512), so a whole 128-column score row stays in registers.  The
+// launcher checks the compiled count before the first launch, because a split larger than
+// the launch allocation would wait forever.
 // The visited KV tiles come from the planner (sink tiles, interval_g tiles, near-diagonal
 // band, merged); only tiles that are not entirely visible apply the element mask.
-// Online softmax in the log2 domain with a lazy rescale of O (only when the running max
-// grows by more than 2^8), P rounded to bf16 into a 128-byte-swizzled shared tile, fp32
-// accumulation throughout.  Epilogue: O / l -> bf16 o, lse = ln(sum exp) in fp32.
 //
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
+// Softmax: online, in the log2 domain, with a lazy rescale of O (only when the running max
+// grows by more than 2^8; the final division uses the same stale max, so the result is
+// exact).  P is rounded to bf16 and written back into TMEM over the S columns it came from,
+// where the P V MMA reads it as its A operand (no shared-memory round trip).  Three of every
+// eight exponentials run as a polynomial on the FMA pipe (exp2_poly.cuh) to balance the
+// special-function unit against the FMA pipe.  fp32 accumulation throughout.
+//
+// MMA order per KV tile n: S0(n), PV1(n-1), S1(n), PV0(n).  Softmax 0 works on S0(n) while
+// the tensor core runs PV1(n-1) and S1(n), softmax 1 on S1(n) during PV0(n) and S0(n+1).
+// tcgen05 MMAs of one thread execute in issue order, so S_k(n+1) overwriting P_k(n) is safe
+// once PV_k(n) is issued, and the commit that announces S_k(n) also covers PV_k(n-1).
+//
+// TMEM (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256, 256+D), O1 [256+D, 256+2D).
 #include <cuda_bf16.h>
 #include <math.h>
 
 #include "cowa_internal.h"
+#include "exp2_poly.cuh"
 #include "kernel_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -27,31 +43,35 @@ namespace cowa {
 namespace {
 
 constexpr int kBM = kTile, kBN = kTile;
-constexpr int kFwdThreads = 320;
-constexpr int kRing = 3;
+constexpr int kFwdThreads = 384;
+constexpr int kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kFwdThreads * kRegsLaunch,
+              "register split must add up to the launch allocation");
+constexpr int kRing = 4;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct FwdGeom {
-  static constexpr int kQBytes = kBM * D * 2;     // one head's Q tile
-  static constexpr int kKVBytes = kBN * D * 2;    // one K or V tile
-  static constexpr int kPBytes = kBM * kBN * 2;   // one head's P tile
+  static constexpr int kQBytes = kBM * D * 2;   // one head's Q tile
+  static constexpr int kKVBytes = kBN * D * 2;  // one K or V tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kQBytes;
-  static constexpr int kOffP = kOffRing + kRing * kKVBytes;
-  static constexpr int kSmem = kOffP + 2 * kPBytes + 1024;  // + alignment slack
+  static constexpr int kSmem = kOffRing + kRing * kKVBytes + 1024;  // + alignment slack
   static constexpr int kColO = 256;
 };
+
+// exponentials of columns c with (c & 7) in {1, 4, 6} go to the FMA pipe
+__device__ __forceinline__ constexpr bool poly_col(int c) { return ((0x52 >> (c & 7)) & 1) != 0; }
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_constant__ FwdArgs a) {
   using Geo = FwdGeom<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align1024(smem_raw);
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t kv_full[kRing], kv_empty[kRing];
-  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_ready[2], o_done[2];
+  __shared__ __align__(8) uint64_t s_full[2], p_ready[2], o_done[2];
   __shared__ __align__(8) uint64_t mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -76,14 +96,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
 
   uint8_t* sQ = smem + Geo::kOffQ;
   uint8_t* sRing = smem + Geo::kOffRing;
-  uint8_t* sP = smem + Geo::kOffP;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 1);
     for (int s = 0; s < kRing; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&s_full[k], 1);
-      ptx::mbar_init(&s_free[k], 4);
       ptx::mbar_init(&p_ready[k], 4);
       ptx::mbar_init(&o_done[k], 1);
     }
@@ -100,7 +118,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const int ntiles = T.count;
-
+  if (warp >= 8) {
+    // warpgroup-wide register reallocation: this warpgroup gives registers to the softmax ones
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+  }
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -136,7 +157,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ), ring_addr = ptx::smem_u32(sRing), p_addr = ptx::smem_u32(sP);
+      const uint32_t q_addr = ptx::smem_u32(sQ), ring_addr = ptx::smem_u32(sRing);
       const int nslot = has1 ? 2 : 1;
 
       auto issue_s = [&](int k, int kslot) {
@@ -148,15 +169,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
                            ptx::smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
+      // O_k (+)= P_k V: P_k (bf16, in TMEM over the S_k columns) is the A operand
       auto issue_pv = [&](int k, int vslot, bool accumulate) {
-        const uint32_t pa = p_addr + k * Geo::kPBytes, vb = ring_addr + vslot * Geo::kKVBytes;
+        const uint32_t vb = ring_addr + vslot * Geo::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + Geo::kColO + k * D, ptx::smem_desc_sw128(pa + aoff, 16, 1024),
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColO + k * D, tmem + k * 128 + kk * 8,
                            ptx::smem_desc_sw128(vb + kk * 2048, 16384, 1024), idesc_o,
                            (accumulate || kk > 0) ? 1u : 0u);
-        }
       };
 
       bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
@@ -166,9 +186,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         const int kslot = kidx % kRing, vslot = vidx % kRing;
         if (!(ok = ptx::mbar_wait(&kv_full[kslot], (kidx / kRing) & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
-        // S0(n)
-        if (n > 0 && !(ok = ptx::mbar_wait(&s_free[0], (n - 1) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
+        // S0(n): P0(n-1) was consumed by PV0(n-1), issued earlier
         issue_s(0, kslot);
         ptx::mma_commit(&s_full[0]);
         if (nslot == 2) {
@@ -178,12 +196,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
             if (!(ok = ptx::mbar_wait(&p_ready[1], (n - 1) & 1, &abort_flag, a.status))) break;
             ptx::tc_fence_after();
             issue_pv(1, pv % kRing, n - 1 > 0);
-            ptx::mma_commit(&o_done[1]);
             ptx::mma_commit(&kv_empty[pv % kRing]);
           }
-          // S1(n)
-          if (n > 0 && !(ok = ptx::mbar_wait(&s_free[1], (n - 1) & 1, &abort_flag, a.status))) break;
-          ptx::tc_fence_after();
           issue_s(1, kslot);
           ptx::mma_commit(&s_full[1]);
         }
@@ -193,24 +207,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         if (!(ok = ptx::mbar_wait(&p_ready[0], n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
         issue_pv(0, vslot, n > 0);
-        ptx::mma_commit(&o_done[0]);
         if (nslot == 1) ptx::mma_commit(&kv_empty[vslot]);
       }
-      if (ok && nslot == 2 && ntiles > 0) {
-        const int n = ntiles - 1, pv = 2 * n + 1;
-        if (ptx::mbar_wait(&p_ready[1], n & 1, &abort_flag, a.status)) {
-          ptx::tc_fence_after();
-          issue_pv(1, pv % kRing, n > 0);
-          ptx::mma_commit(&o_done[1]);
-          ptx::mma_commit(&kv_empty[pv % kRing]);
+      if (ok && ntiles > 0) {
+        ptx::mma_commit(&o_done[0]);
+        if (nslot == 2) {
+          const int n = ntiles - 1, pv = 2 * n + 1;
+          if (ptx::mbar_wait(&p_ready[1], n & 1, &abort_flag, a.status)) {
+            ptx::tc_fence_after();
+            issue_pv(1, pv % kRing, n > 0);
+            ptx::mma_commit(&kv_empty[pv % kRing]);
+            ptx::mma_commit(&o_done[1]);
+          }
         }
       }
       // all issued MMAs complete before TMEM can be released
       ptx::mma_commit(&mma_final);
       ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int k = warp >> 2;  // head slot
     if (k == 0 || has1) {
       const int r = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
@@ -218,9 +235,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
       const uint32_t s_tm = lane_base + k * 128;
       const uint32_t o_tm = lane_base + Geo::kColO + k * D;
-      uint8_t* prow = sP + k * Geo::kPBytes + r * 128;
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = -INFINITY;
       const float sl2 = a.scale_log2;
+      const uint64_t sl2x2 = ptx::f2_pack(sl2, sl2);
+      uint64_t lsum = ptx::f2_pack(0.f, 0.f);
       bool ok = true;
       TileCursor cur;
       cur.init(T);
@@ -229,46 +247,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         const bool need_mask = (s0 + kBN > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kBN));
         if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
-        uint32_t sr[128];
+        uint32_t xr[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(s_tm + c * 32, sr + c * 32);
+        for (int q = 0; q < 4; ++q) ptx::tmem_ld32(s_tm + q * 32, xr + q * 32);
         ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&s_free[k]);
-
-        float x[128];
-        float mx = -INFINITY;
+        // visible key columns of row t within [s0, s0+128), relative to s0 (partial tiles only)
+        const int sink_end = imin(a.pat.S, t + 1) - s0;
+        const int band_lo = imax(0, t - a.pat.L + 1) - s0;
+        const int diag_end = t + 1 - s0;
+        const int lr_lo = iv.lo - s0, lr_hi = imin(iv.hi, t + 1) - s0;
         if (need_mask) {
-          // visible key columns of row t within [s0, s0+128), relative to s0
-          const int sink_end = imin(a.pat.S, t + 1) - s0;
-          const int band_lo = imax(0, t - a.pat.L + 1) - s0;
-          const int diag_end = t + 1 - s0;
-          const int lr_lo = iv.lo - s0, lr_hi = imin(iv.hi, t + 1) - s0;
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const bool vis = (c < sink_end) || (c >= band_lo && c < diag_end) || (c >= lr_lo && c < lr_hi);
-            x[c] = vis ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] = __uint_as_float(sr[c]) * sl2;
-            mx = fmaxf(mx, x[c]);
+            if (!vis) xr[c] = 0xff800000u;  // -inf
           }
         }
-        const float m_new = fmaxf(m_used, mx);
-        // the previous PV of this head must be done before P is overwritten / O rescaled
-        if (n > 0 && !(ok = ptx::mbar_wait_warp(&o_done[k], (n - 1) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        // lazy rescale: only when the running max grows by more than 2^8 (or first finite max)
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) mx = ptx::fmax3(mx, __uint_as_float(xr[c]), __uint_as_float(xr[c + 1]));
+        const float m_new = fmaxf(m_used, mx * sl2);
+        // lazy rescale: only when the running max grows by more than 2^8 (or first finite max);
+        // PV_k(n-1) has completed (the commit of S_k(n) covers it), so O_k is stable here
         const bool grow = (m_new != -INFINITY) && (m_used == -INFINITY || m_new > m_used + kRescaleThreshold);
         float alpha = 1.f;
         if (grow) {
           alpha = ptx::ex2(m_used - m_new);  // 0 when nothing was visible before
-          l *= alpha;
           m_used = m_new;
+          lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
         }
         if (n > 0 && __any_sync(0xffffffffu, grow)) {
           // O row *= alpha, a warp-collective TMEM round trip (alpha = 1 on the other lanes)
@@ -281,51 +287,64 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
             ptx::tmem_st32(o_tm + c * 32, ov);
           }
-          ptx::tmem_wait_st();
         }
         const float m_eff = m_used == -INFINITY ? 0.f : m_used;
-        float rowsum = 0.f;
+        const uint64_t negm = ptx::f2_pack(-m_eff, -m_eff);
+        // P = 2^(s*scale*log2e - m), rounded to bf16, back into TMEM over the S columns
+        // (masked scores are -inf and give exactly 0)
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {
-          uint32_t w[4];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pw[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ptx::ex2(x[c8 * 8 + 2 * e] - m_eff);
-            const float p1 = ptx::ex2(x[c8 * 8 + 2 * e + 1] - m_eff);
-            rowsum += p0 + p1;
-            w[e] = ptx::pack_bf16(p0, p1);
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const int c = 64 * h + 2 * c2;
+            float e0, e1;
+            ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), sl2x2, negm),
+                           e0, e1);
+            float p0, p1;
+            if (need_mask) {
+              p0 = ptx::ex2(e0);
+              p1 = ptx::ex2(e1);
+            } else {
+              p0 = poly_col(c) ? exp2_fma(e0) : ptx::ex2(e0);
+              p1 = poly_col(c + 1) ? exp2_fma(e1) : ptx::ex2(e1);
+            }
+            lsum = ptx::f2_add(lsum, ptx::f2_pack(p0, p1));
+            pw[c2] = ptx::pack_bf16(p0, p1);
           }
-          const int chunk = c8 >> 3, unit = c8 & 7;
-          uint4* dst = reinterpret_cast<uint4*>(prow + chunk * 16384 + ((unit ^ (r & 7)) << 4));
-          *dst = make_uint4(w[0], w[1], w[2], w[3]);
+          ptx::tmem_st32(s_tm + 32 * h, pw);
         }
-        l += rowsum;
-        ptx::fence_proxy_async_smem();
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&p_ready[k]);
       }
+      float la, lb;
+      ptx::f2_unpack(lsum, la, lb);
+      const float l = la + lb;
       // ---- epilogue
-      if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], (ntiles - 1) & 1, &abort_flag, a.status)) {
+      if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], 0, &abort_flag, a.status)) {
         ptx::tc_fence_after();
-        uint32_t ov[D];
+        const float inv = 1.f / l;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)t * a.o_st +
+                              (size_t)(h0 + k) * a.o_sh;
+        if (t < a.N) a.lse[((size_t)b * a.Hq + h0 + k) * a.N + t] = (m_used + log2f(l)) * 0.69314718055994530942f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(o_tm + c * 32, ov + c * 32);
-        ptx::tmem_wait_ld();
-        if (t < a.N) {
-          const float inv = 1.f / l;
-          __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)t * a.o_st +
-                                (size_t)(h0 + k) * a.o_sh;
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(o_tm + c * 32, ov);  // warp-collective: every lane loads, valid rows store
+          ptx::tmem_wait_ld();
+          if (t < a.N) {
 #pragma unroll
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            uint32_t w[4];
+            for (int c8 = 0; c8 < 4; ++c8) {
+              uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = ptx::pack_bf16(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv,
-                                    __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv);
-            reinterpret_cast<uint4*>(orow)[c8] = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int e = 0; e < 4; ++e)
+                w[e] = ptx::pack_bf16(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv,
+                                      __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv);
+              reinterpret_cast<uint4*>(orow)[c * 4 + c8] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
-          a.lse[((size_t)b * a.Hq + h0 + k) * a.N + t] = (m_used + log2f(l)) * 0.69314718055994530942f;
         }
       }
     }
@@ -349,6 +368,14 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   const int nq = (a.N + kBM - 1) / kBM;
   const long long nblk = (long long)nq * a.B * a.Hkv * ((grp + 1) / 2);
   if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
+  // the in-kernel register split assumes the compiled count equals the launch allocation
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    regs_ok = fa.numRegs == kRegsLaunch ? 1 : 0;
+  }
+  if (!regs_ok) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)nblk, kFwdThreads, Geo::kSmem, s>>>(a);
   return cudaGetLastError();
 }
