@@ -348,6 +348,9 @@ def run_cowa(args, world, rank, local):
     def fwd():
         cw.cowa_fwd(q, k, v, pat, out=o, lse=lse, workspace=ws_f)
 
+    def bwd_stage(st):
+        cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws_b, stages=st)
+
     def bwd():
         cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws_b)
 
@@ -366,23 +369,30 @@ def run_cowa(args, world, rank, local):
         fwd(); bwd(); dec()
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, events between the three calls
+    # ---- timed region: K steps, events between the calls (the backward as its three stages,
+    # each one kernel, so that every hot kernel gets its own device time)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         e_start.record()
         for s in range(K):
-            ev[s][0].record(); fwd(); ev[s][1].record(); bwd(); ev[s][2].record(); dec(); ev[s][3].record()
+            e = ev[s]
+            e[0].record(); fwd()
+            e[1].record(); bwd_stage(cw.BWD_PREPROCESS)
+            e[2].record(); bwd_stage(cw.BWD_DKDV)
+            e[3].record(); bwd_stage(cw.BWD_DQ)
+            e[4].record(); dec()
+            e[5].record()
         e_end.record()
         torch.cuda.synchronize()
         barrier()
     total_ms = maxr(e_start.elapsed_time(e_end))
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    dec_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    avg = lambda a_, b_: statistics.mean(e[a_].elapsed_time(e[b_]) for e in ev)
+    fwd_ms, pre_ms, dkdv_ms, dq_ms, dec_ms = avg(0, 1), avg(1, 2), avg(2, 3), avg(3, 4), avg(4, 5)
+    bwd_ms = pre_ms + dkdv_ms + dq_ms
     for st in (cw.workspace_status(ws_f), cw.workspace_status(ws_b), cw.workspace_status(ws_d)):
         if st != 0:
             raise RuntimeError(f"device status {st} after the timed region")
@@ -398,7 +408,8 @@ def run_cowa(args, world, rank, local):
     burst, sustained, hbm, peak_src = _peaks()
     parts = {
         "fwd": {"ms": fwd_ms, "tflops_visible": fwd_flop / (fwd_ms * 1e-3) / 1e12},
-        "bwd": {"ms": bwd_ms, "tflops_visible": bwd_flop / (bwd_ms * 1e-3) / 1e12},
+        "bwd": {"ms": bwd_ms, "tflops_visible": bwd_flop / (bwd_ms * 1e-3) / 1e12,
+                "stages_ms": {"preprocess": pre_ms, "dkdv": dkdv_ms, "dq": dq_ms}},
         "decode": {"ms": dec_ms, "gbs_visible": dec_bytes / (dec_ms * 1e-3) / 1e9,
                    "frac_hbm": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "visible_bytes": dec_bytes},
     }
@@ -420,12 +431,30 @@ def run_cowa(args, world, rank, local):
         parts["fwd_dense_causal"] = {"ms": dms, "tflops": 4.0 * c["d"] * dpairs / (dms * 1e-3) / 1e12,
                                      "speedup_cowa_vs_dense": dms / fwd_ms}
 
-    # ---- roofline of the dominant kernel: the forward kernel is one launch per cowa_fwd
-    fwd_traffic = _traffic_record("cowa_fwd.cu")
-    roofline = {"kernel": "cowa_fwd_kernel<128>", "bound": "tensor", "achieved": parts["fwd"]["tflops_visible"],
-                "peak": sustained, "unit": "TFLOP/s", "frac": parts["fwd"]["tflops_visible"] / sustained,
-                "traffic": fwd_traffic, "peak_source": f"{peak_src} bf16 sustained",
-                "algorithmic": f"{fwd_flop:.4e} FLOP per launch = 4*d*visible pairs ({pairs:.4e})"}
+    # ---- roofline of the dominant kernel (longest device time in the step).  Algorithmic work per
+    # launch: forward 2 GEMMs (4*d per visible pair), dK/dV 4 GEMMs (S^T, dP^T, dV, dK: 8*d per
+    # pair), dQ 3 GEMMs (S, dP, dQ: 6*d per pair), decode the visible K/V bytes once.
+    kernels = {
+        "cowa_fwd_kernel<128>": (fwd_ms, fwd_flop, "tensor", "cowa_fwd.cu", "4*d"),
+        "bwd_dkdv_kernel<128>": (dkdv_ms, 8.0 * c["d"] * pairs, "tensor", "cowa_bwd.cu", "8*d"),
+        "bwd_dq_kernel<128>": (dq_ms, 6.0 * c["d"] * pairs, "tensor", "cowa_bwd.cu", "6*d"),
+        "decode_split_kernel<5,128>": (dec_ms, dec_bytes, "hbm", "cowa_decode.cu", None),
+    }
+    top = max(kernels, key=lambda kname: kernels[kname][0])
+    t_ms, work, bound, src, per = kernels[top]
+    if bound == "tensor":
+        achieved = work / (t_ms * 1e-3) / 1e12
+        roofline = {"kernel": top, "bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                    "frac": achieved / sustained, "traffic": _traffic_record(src),
+                    "peak_source": f"{peak_src} bf16 dense, sustained",
+                    "algorithmic": f"{work:.4e} FLOP per launch = {per} x visible pairs ({pairs:.4e})"}
+    else:
+        achieved = work / (t_ms * 1e-3) / 1e9
+        roofline = {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "traffic": _traffic_record(src),
+                    "peak_source": f"{peak_src} HBM copy",
+                    "algorithmic": f"{work:.4e} visible K/V bytes per call"}
+    roofline["all_kernels_ms"] = {kname: v[0] for kname, v in kernels.items()}
 
     # ---- end to end: host buffers, copies inside the timed region
     e2e = None
@@ -477,7 +506,7 @@ def run_cowa(args, world, rank, local):
                        "train": TRAIN, "decode": DECODE, "l2": "inputs larger than L2 (126 MB); no flush",
                        "parallelism": f"batch-sharded x{world} (weak)"},
             "parts": parts, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": K * 6, "clocks": clk.summary()}
+            "gpu_launches": K * 6, "clocks": clk.summary()}  # fwd 1 + bwd 3 + decode 2 per step
     print(json.dumps(line), flush=True)
     return 0
 

@@ -108,6 +108,20 @@ cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, i
                      cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* Backward in stages.  `stages` is a bit mask of COWA_BWD_PREPROCESS (Delta and lse*log2(e)
+ * into the workspace), COWA_BWD_DKDV (dk, dv) and COWA_BWD_DQ (dq); cowa_bwd is all three.
+ * The dK/dV and dQ stages read what the preprocess stage wrote into the same workspace, so it
+ * must have completed first (stream order); they are independent of each other and may run on
+ * two streams that both wait for the preprocess.  Arguments are those of cowa_bwd; a stage
+ * outside the mask does not touch its outputs. */
+#define COWA_BWD_PREPROCESS 1
+#define COWA_BWD_DKDV 2
+#define COWA_BWD_DQ 4
+cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d,
+                            cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse,
+                            cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
+                            int stages, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- decode (one new token per sequence, KV cache) -----------------------------------------
  * q_t    [B, H_q, d] bf16, contiguous.
  * k_cache, v_cache: cowa_tensor over [B, T_cap, H_kv, d]-indexed (b, t, h) with any strides
@@ -169,6 +183,13 @@ const char* cowa_status_string(cowa_status s);
 cowa_status cowa_visible_counts(const cowa_pattern* pat, int H_kv, int N, int64_t* out);
 cowa_status cowa_plan_debug(const cowa_pattern* pat, int H_kv, int N, int BM, int BN, int which,
                             int32_t* out, size_t cap, size_t* n_written, void* dev_scratch);
+
+/* Test hook for the failure path every kernel's device-side waits share: launches one CTA that
+ * waits on a barrier nothing arrives on.  After limit_ns (1 us .. 10 s) the wait gives up, the
+ * timeout is recorded in the status word of `ws` (>= 256 bytes) and the kernel returns; a
+ * following cowa_workspace_status(ws, stream) reports COWA_ERR_TIMEOUT and the context stays
+ * usable.  No fault, trap or hang is involved. */
+cowa_status cowa_debug_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream);
 
 int cowa_version(void);
 

@@ -27,7 +27,9 @@ _STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED", 3
 
 EXPORTED = ["cowa_fwd_workspace_size", "cowa_fwd", "cowa_bwd_workspace_size", "cowa_bwd",
             "cowa_decode_workspace_size", "cowa_decode", "cowa_workspace_status", "cowa_status_string",
-            "cowa_visible_counts", "cowa_plan_debug", "cowa_version", "cowa_decode_noalloc"]
+            "cowa_visible_counts", "cowa_plan_debug", "cowa_version", "cowa_decode_noalloc", "cowa_bwd_stages", "cowa_debug_wait_timeout"]
+
+BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 1, 2, 4
 
 
 class CowaError(RuntimeError):
@@ -84,6 +86,8 @@ def lib() -> ctypes.CDLL:
     L.cowa_bwd_workspace_size.restype = sz
     L.cowa_bwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
     L.cowa_bwd.restype = i
+    L.cowa_bwd_stages.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, i, vp, sz, vp]
+    L.cowa_bwd_stages.restype = i
     L.cowa_decode_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_decode_workspace_size.restype = sz
     L.cowa_decode.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp, sz, vp]
@@ -98,6 +102,8 @@ def lib() -> ctypes.CDLL:
     L.cowa_visible_counts.restype = i
     L.cowa_plan_debug.argtypes = [P, i, i, i, i, i, vp, sz, ctypes.POINTER(sz), vp]
     L.cowa_plan_debug.restype = i
+    L.cowa_debug_wait_timeout.argtypes = [vp, sz, ctypes.c_int64, vp]
+    L.cowa_debug_wait_timeout.restype = i
     L.cowa_version.argtypes = []
     L.cowa_version.restype = i
     _lib = L
@@ -158,8 +164,10 @@ def cowa_fwd(q, k, v, pattern: Pattern, out=None, lse=None, workspace=None, stre
     return out, lse
 
 
-def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """(dq, dk, dv) bf16: gradients of sum(do * o) for the forward with the same inputs."""
+def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, workspace=None, stream=None,
+             stages: int = 7):
+    """(dq, dk, dv) bf16: gradients of sum(do * o) for the forward with the same inputs.
+    `stages` selects BWD_PREPROCESS | BWD_DKDV | BWD_DQ (all by default)."""
     import torch
 
     for n_, x_ in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
@@ -174,9 +182,15 @@ def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, w
     ws_bytes = L.cowa_bwd_workspace_size(ctypes.byref(pat), B, N, Hq, Hkv, d)
     if workspace is None:
         workspace = _workspace(ws_bytes, q.device)
-    _check("cowa_bwd", L.cowa_bwd(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v), _t4(o),
-                                  lse.data_ptr(), _t4(do), _t4(dq), _t4(dk), _t4(dv),
-                                  workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    if stages == 7:
+        _check("cowa_bwd", L.cowa_bwd(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v), _t4(o),
+                                      lse.data_ptr(), _t4(do), _t4(dq), _t4(dk), _t4(dv),
+                                      workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    else:
+        _check("cowa_bwd_stages", L.cowa_bwd_stages(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v),
+                                                    _t4(o), lse.data_ptr(), _t4(do), _t4(dq), _t4(dk), _t4(dv),
+                                                    stages, workspace.data_ptr(), workspace.numel(),
+                                                    _stream(stream)))
     return dq, dk, dv
 
 

@@ -100,6 +100,15 @@ extern "C" {
 
 int cowa_version(void) { return 1; }
 
+cowa_status cowa_debug_wait_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream) {
+  COWA_TRY(check_ws(ws, ws_bytes, kWsHeader));
+  if (limit_ns < 1000 || limit_ns > 10000000000LL) return COWA_ERR_INVALID_ARG;
+  return launch_wait_timeout_probe(reinterpret_cast<uint32_t*>(ws), (unsigned long long)limit_ns,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
+}
+
 const char* cowa_status_string(cowa_status s) {
   switch (s) {
     case COWA_OK: return "ok";
@@ -210,6 +219,15 @@ size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int Hq, in
 cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d, cowa_tensor q, cowa_tensor k,
                      cowa_tensor v, cowa_tensor o, const float* lse, cowa_tensor dO, cowa_tensor dq, cowa_tensor dk,
                      cowa_tensor dv, void* ws, size_t ws_bytes, void* stream) {
+  return cowa_bwd_stages(pat, B, N, Hq, Hkv, d, q, k, v, o, lse, dO, dq, dk, dv,
+                         COWA_BWD_PREPROCESS | COWA_BWD_DKDV | COWA_BWD_DQ, ws, ws_bytes, stream);
+}
+
+cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d, cowa_tensor q,
+                            cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse, cowa_tensor dO,
+                            cowa_tensor dq, cowa_tensor dk, cowa_tensor dv, int stages, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (stages <= 0 || stages > (COWA_BWD_PREPROCESS | COWA_BWD_DKDV | COWA_BWD_DQ)) return COWA_ERR_INVALID_ARG;
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
   COWA_TRY(check_heads(B, N, Hq, Hkv, d));
@@ -239,7 +257,7 @@ cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int
       !make_tmap_bf16(&a.tm_v, v.ptr, d, N, Hkv, B, v.stride_t, v.stride_h, v.stride_b, 128) ||
       !make_tmap_bf16(&a.tm_do, dO.ptr, d, N, Hq, B, dO.stride_t, dO.stride_h, dO.stride_b, 128))
     return COWA_ERR_CUDA;
-  return launch_bwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+  return launch_bwd(a, stages, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------------ introspection

@@ -14,14 +14,17 @@
 //      every query head of the group.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the
 //      elementwise softmax writes P^T and dS^T back into TMEM as bf16, where they are the A
 //      operand of dV += P^T dO and dK += dS^T Q (tcgen05 MMA with A in TMEM);
-//   3. dQ: one CTA per (b, query head h, 128-row tile i) over the forward tile plan; S and
-//      dP in TMEM, dS back into TMEM as bf16, dQ += dS K with A in TMEM.
+//   3. dQ: one CTA per (b, query head h, 128-row tile i) over the forward tile plan.  The
+//      softmax warps load S and dP of a KV tile into registers and release them at once, so
+//      the MMA warp computes S and dP of the next tile while dS of this one is being formed;
+//      dS goes to a double-buffered bf16 region of TMEM and dQ += dS K reads it as A.
 // Warp roles in both attention kernels: warps 0-7 elementwise softmax (two warps per TMEM
 // lane quadrant, each owning half of the columns), warp 8 TMA producer, warp 9 MMA issuer.
 #include <cuda_bf16.h>
 #include <math.h>
 
 #include "cowa_internal.h"
+#include "exp2_poly.cuh"
 #include "kernel_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -32,6 +35,19 @@ constexpr int kThreads = 320;
 constexpr int kComputeWarps = 8;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kStatBytes = 1024;  // lse2[128] + delta[128] of one query tile
+
+// Which exponentials run on the FMA pipe (exp2_poly.cuh) instead of the special-function unit:
+// column c goes to the FMA pipe when bit (c & 7) of the kernel's mask is set.  Both backward
+// softmaxes are bound by instruction issue rather than by the special-function unit on B200
+// (measured: every offloaded share was slower), so the masks default to 0.
+#ifndef COWA_DKDV_POLY_MASK
+#define COWA_DKDV_POLY_MASK 0x00
+#endif
+#ifndef COWA_DQ_POLY_MASK
+#define COWA_DQ_POLY_MASK 0x00
+#endif
+template <int MASK>
+__device__ __forceinline__ constexpr bool poly_col(int c) { return ((MASK >> (c & 7)) & 1) != 0; }
 
 template <int D>
 struct BwdGeom {
@@ -228,15 +244,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&ld_done);
       const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes);
+      // all lanes read the same statistics: 16-byte broadcast loads
+      const float4* lse4 = reinterpret_cast<const float4*>(stat + half * 64);
+      const float4* del4 = reinterpret_cast<const float4*>(stat + 128 + half * 64);
+      const bool use_poly = !need_mask && t0 + kTile <= a.N;
       float pf[64], df[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int col = half * 64 + c;
-        const int t = t0 + col;
-        float p = ptx::ex2(__uint_as_float(sv[c]) * sl2 - stat[col]);
-        if (need_mask && !(t >= s && t < t_hi)) p = 0.f;
-        pf[c] = p;
-        df[c] = p * (__uint_as_float(pv[c]) - stat[128 + col]);
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 ls = lse4[c4], dl = del4[c4];
+        const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c4 * 4 + e;
+          const float x = fmaf(__uint_as_float(sv[c]), sl2, -lsv[e]);
+          float p = (use_poly && poly_col<COWA_DKDV_POLY_MASK>(c)) ? exp2_fma(x) : ptx::ex2(x);
+          if (need_mask) {
+            const int t = t0 + half * 64 + c;
+            if (!(t >= s && t < t_hi)) p = 0.f;
+          }
+          pf[c] = p;
+          df[c] = p * (__uint_as_float(pv[c]) - dlv[e]);
+        }
       }
       uint32_t pw[32], dw[32];
       pack64(pf, pw);
@@ -291,12 +319,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
 }
 
 // ------------------------------------------------------------------------------ dQ
+// TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D), dS double buffer 2 x 64 after dQ.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
   using Geo = BwdGeom<D>;
+  constexpr uint32_t kColDS = Geo::kColAcc + D;  // first dS buffer
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], sdp_full, ld_done, p_ready, acc_full, mma_final;
+  // ds_ready is per dS buffer: a barrier can then never run two phases ahead of its waiter
+  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], sdp_full, consumed, ds_ready[2], acc_full,
+      mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -321,8 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     ptx::mbar_init(&q_full, 1);
     for (int s = 0; s < 2; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
     ptx::mbar_init(&sdp_full, 1);
-    ptx::mbar_init(&ld_done, kComputeWarps);
-    ptx::mbar_init(&p_ready, kComputeWarps);
+    ptx::mbar_init(&consumed, kComputeWarps);
+    ptx::mbar_init(&ds_ready[0], kComputeWarps);
+    ptx::mbar_init(&ds_ready[1], kComputeWarps);
     ptx::mbar_init(&acc_full, 1);
     ptx::mbar_init(&mma_final, 1);
     abort_flag = 0;
@@ -369,13 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
       const uint32_t q_addr = ptx::smem_u32(sQ), do_addr = ptx::smem_u32(sDO), slot_addr = ptx::smem_u32(sSlot);
-      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
-      ptx::tc_fence_after();
-      for (int n = 0; ok && n < ntiles; ++n) {
-        const int slot = n & 1;
-        const uint32_t ka = slot_addr + slot * Geo::kSlotQ, va = ka + Geo::kTileBytes;
-        if (!(ok = ptx::mbar_wait(&kv_full[slot], (n >> 1) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
+      // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns
+      auto issue_sdp = [&](int n) {
+        const uint32_t ka = slot_addr + (n & 1) * Geo::kSlotQ, va = ka + Geo::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -389,14 +418,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
                            ptx::smem_desc_sw128(va + off, 16, 1024), idesc_s, kk > 0);
         }
         ptx::mma_commit(&sdp_full);
-        if (!(ok = ptx::mbar_wait(&p_ready, n & 1, &abort_flag, a.status))) break;
+      };
+      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
+      ptx::tc_fence_after();
+      if (ok && ntiles > 0 && (ok = ptx::mbar_wait(&kv_full[0], 0, &abort_flag, a.status))) {
         ptx::tc_fence_after();
-        // dQ += dS K : A = dS in TMEM, B = K MN-major in smem
+        issue_sdp(0);
+      }
+      for (int n = 0; ok && n < ntiles; ++n) {
+        // the softmax holds S(n), dP(n) in registers: compute the next tile's S and dP now
+        if (!(ok = ptx::mbar_wait(&consumed, n & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        if (n + 1 < ntiles) {
+          if (!(ok = ptx::mbar_wait(&kv_full[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, a.status))) break;
+          ptx::tc_fence_after();
+          issue_sdp(n + 1);
+        }
+        if (!(ok = ptx::mbar_wait(&ds_ready[n & 1], (n >> 1) & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        // dQ += dS K : A = dS (TMEM buffer n & 1), B = K MN-major in smem
+        const uint32_t ka = slot_addr + (n & 1) * Geo::kSlotQ;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + 0 + kk * 8, ptx::smem_desc_sw128(ka + kk * 2048, 16384, 1024),
-                           idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(&kv_empty[slot]);
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + kColDS + (n & 1) * 64 + kk * 8,
+                           ptx::smem_desc_sw128(ka + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(&kv_empty[n & 1]);
       }
       if (ok) ptx::mma_commit(&acc_full);
       ptx::mma_commit(&mma_final);
@@ -430,27 +476,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&ld_done);
-      float df[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int s = s0 + half * 64 + c;
-        float p = ptx::ex2(__uint_as_float(sv[c]) * sl2 - lse2);
-        if (need_mask) {
-          const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
-          if (!vis) p = 0.f;
-        }
-        df[c] = p * (__uint_as_float(pv[c]) - delta);
-      }
+      if (lane == 0) ptx::mbar_arrive(&consumed);  // S / dP columns may be overwritten now
+      const bool use_poly = !need_mask && t < a.N;
       uint32_t dw[32];
-      pack64(df, dw);
-      if (!(ok = ptx::mbar_wait_warp(&ld_done, n & 1, &abort_flag, a.status))) break;
-      ptx::tc_fence_after();
-      ptx::tmem_st32(lane_base + half * 32, dw);
+#pragma unroll
+      for (int c2 = 0; c2 < 32; ++c2) {
+        float d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 2 * c2 + e;
+          const float x = fmaf(__uint_as_float(sv[c]), sl2, -lse2);
+          float p = (use_poly && poly_col<COWA_DQ_POLY_MASK>(c)) ? exp2_fma(x) : ptx::ex2(x);
+          if (need_mask) {
+            const int s = s0 + half * 64 + c;
+            const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
+            if (!vis) p = 0.f;
+          }
+          d2[e] = p * (__uint_as_float(pv[c]) - delta);
+        }
+        dw[c2] = ptx::pack_bf16(d2[0], d2[1]);
+      }
+      // dS buffer n & 1 was last read by dQ(n-2), which the commit of S(n) covers
+      ptx::tmem_st32(lane_base + kColDS + (n & 1) * 64 + half * 32, dw);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&p_ready);
+      if (lane == 0) ptx::mbar_arrive(&ds_ready[n & 1]);
     }
     if (ok && ntiles > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
       ptx::tc_fence_after();
@@ -484,25 +535,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
+cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
   using Geo = BwdGeom<D>;
   const int nq = a.N_pad / kTile;
-  bwd_preprocess_kernel<D><<<dim3(nq, a.Hq, a.B), 256, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  auto kdkdv = bwd_dkdv_kernel<D>;
-  auto kdq = bwd_dq_kernel<D>;
-  if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemKV)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemQ)) != cudaSuccess)
-    return e;
-  const long long n_kv = (long long)nq * a.Hkv * a.B;
-  const long long n_q = (long long)nq * a.Hq * a.B;
-  if (n_q > 0x7fffffffLL) return cudaErrorInvalidValue;
-  kdkdv<<<(unsigned)n_kv, kThreads, Geo::kSmemKV, s>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kdq<<<(unsigned)n_q, kThreads, Geo::kSmemQ, s>>>(a);
-  return cudaGetLastError();
+  cudaError_t e;
+  if (stages & COWA_BWD_PREPROCESS) {
+    bwd_preprocess_kernel<D><<<dim3(nq, a.Hq, a.B), 256, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (stages & COWA_BWD_DKDV) {
+    auto kdkdv = bwd_dkdv_kernel<D>;
+    if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemKV)) != cudaSuccess)
+      return e;
+    const long long n_kv = (long long)nq * a.Hkv * a.B;
+    if (n_kv > 0x7fffffffLL) return cudaErrorInvalidValue;
+    kdkdv<<<(unsigned)n_kv, kThreads, Geo::kSmemKV, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (stages & COWA_BWD_DQ) {
+    auto kdq = bwd_dq_kernel<D>;
+    if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemQ)) != cudaSuccess)
+      return e;
+    const long long n_q = (long long)nq * a.Hq * a.B;
+    if (n_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+    kdq<<<(unsigned)n_q, kThreads, Geo::kSmemQ, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -513,9 +572,9 @@ size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d) {
   return align_up(2 * (size_t)B * Hq * n_pad * sizeof(float), 256);
 }
 
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t s) {
-  if (a.d == 64) return launch_bwd_d<64>(a, s);
-  if (a.d == 128) return launch_bwd_d<128>(a, s);
+cudaError_t launch_bwd(const BwdArgs& a, int stages, cudaStream_t s) {
+  if (a.d == 64) return launch_bwd_d<64>(a, stages, s);
+  if (a.d == 128) return launch_bwd_d<128>(a, stages, s);
   return cudaErrorInvalidValue;
 }
 

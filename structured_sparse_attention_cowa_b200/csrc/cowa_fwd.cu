@@ -21,9 +21,10 @@
 // Softmax: online, in the log2 domain, with a lazy rescale of O (only when the running max
 // grows by more than 2^8; the final division uses the same stale max, so the result is
 // exact).  P is rounded to bf16 and written back into TMEM over the S columns it came from,
-// where the P V MMA reads it as its A operand (no shared-memory round trip).  Three of every
-// eight exponentials run as a polynomial on the FMA pipe (exp2_poly.cuh) to balance the
-// special-function unit against the FMA pipe.  fp32 accumulation throughout.
+// where the P V MMA reads it as its A operand (no shared-memory round trip).  fp32
+// accumulation throughout.  Exponentials run on the special-function unit; COWA_FWD_POLY_MASK
+// can move a share of them to an FMA-pipe polynomial (exp2_poly.cuh), which measured slower
+// on B200 for this kernel (its softmax is bound by instruction issue), so it is off.
 //
 // MMA order per KV tile n: S0(n), PV1(n-1), S1(n), PV0(n).  Softmax 0 works on S0(n) while
 // the tensor core runs PV1(n-1) and S1(n), softmax 1 on S1(n) during PV0(n) and S0(n+1).
@@ -61,8 +62,12 @@ struct FwdGeom {
   static constexpr int kColO = 256;
 };
 
-// exponentials of columns c with (c & 7) in {1, 4, 6} go to the FMA pipe
-__device__ __forceinline__ constexpr bool poly_col(int c) { return ((0x52 >> (c & 7)) & 1) != 0; }
+// Exponentials of columns c with bit (c & 7) of the mask set go to the FMA pipe (exp2_poly.cuh);
+// e.g. 0x52 = columns 1, 4, 6 of every 8.  Off by default (see above).
+#ifndef COWA_FWD_POLY_MASK
+#define COWA_FWD_POLY_MASK 0x00
+#endif
+__device__ __forceinline__ constexpr bool poly_col(int c) { return ((COWA_FWD_POLY_MASK >> (c & 7)) & 1) != 0; }
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_constant__ FwdArgs a) {

@@ -73,7 +73,10 @@ struct BwdArgs {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
 };
 size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d);
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd(const BwdArgs& a, int stages, cudaStream_t s);
+
+// ---- bounded-wait probe ----
+cudaError_t launch_wait_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t s);
 
 // ---- planner debug kernel ----
 cudaError_t launch_plan_debug(const Pat& p, int Hkv, int N, int BM, int BN, int32_t* dev_out, size_t cap,

@@ -1,7 +1,9 @@
-// cowa_plan.cu -- device-side evaluation of the forward tile plan, for introspection.
-// Runs exactly the planner code (cowa_pattern.h) that the attention kernels run on the
-// fly, so a host test can compare the device plan with the host plan and the mask.
+// cowa_plan.cu -- device-side evaluation of the forward tile plan, for introspection, and the
+// bounded-wait probe.  The plan kernel runs exactly the planner code (cowa_pattern.h) that the
+// attention kernels run on the fly, so a host test can compare the device plan with the host
+// plan and the mask.  The probe kernel exercises the timeout path every kernel's waits share.
 #include "cowa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace cowa {
 namespace {
@@ -27,7 +29,24 @@ __global__ void plan_debug_kernel(Pat p, int Hkv, int N, int BM, int BN, int32_t
   }
 }
 
+// One thread waits on an mbarrier that nothing will ever arrive on.  The wait gives up after
+// limit_ns, records the timeout in the status word and the kernel returns normally.
+__global__ void wait_timeout_probe_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  ptx::mbar_init(&bar, 1);
+  ptx::fence_mbar_init();
+  ptx::mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_probe(uint32_t* status, unsigned long long limit_ns, cudaStream_t s) {
+  wait_timeout_probe_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_plan_debug(const Pat& p, int Hkv, int N, int BM, int BN, int32_t* dev_out, size_t cap,
                               unsigned long long* dev_count, cudaStream_t s) {

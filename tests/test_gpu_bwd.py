@@ -110,5 +110,30 @@ def test_bwd_long_128k(cuda_device):
     columns and the any-size identities."""
     pat = cw.Pattern(128, 4096, 131072, 8)
     rows = np.array([0, 127, 128, 4095, 4096, 16495, 16496, 70000, 131071])
-    _check_sampled(1, 131072, 40, 8, 128, pat, cuda_device, rows, [(3, [20000, 50001]), (7, [131071])],
+    _check_sampled(1, 131072, 40, 8, 128, pat, cuda_device, rows, [(3, [20000, 40001]), (7, [131071])],
                    cuda_gen=True)
+
+
+def test_bwd_stages_on_two_streams_match_single_call(cuda_device):
+    """The staged entry point: preprocess, then dK/dV and dQ on two streams that both wait for
+    it, gives the same bits as one cowa_bwd call (the kernels are deterministic)."""
+    B, N, Hq, Hkv, d = 1, 1500, 10, 2, 128
+    pat = cw.Pattern(64, 200, 1500, 2)
+    _, (q, k, v, do) = _inputs(B, N, Hq, Hkv, d, cuda_device, extra=9)
+    o, lse = cw.cowa_fwd(q, k, v, pat)
+    dq1, dk1, dv1 = cw.cowa_bwd(q, k, v, o, lse, do, pat)
+    import ctypes
+    n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+    ws = torch.zeros(n, dtype=torch.uint8, device=cuda_device)
+    dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    main = torch.cuda.current_stream()
+    cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq2, dk=dk2, dv=dv2, workspace=ws, stages=cw.BWD_PREPROCESS)
+    ev = torch.cuda.Event()
+    ev.record(main)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    s1.wait_event(ev)
+    s2.wait_event(ev)
+    cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq2, dk=dk2, dv=dv2, workspace=ws, stages=cw.BWD_DKDV, stream=s1)
+    cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq2, dk=dk2, dv=dv2, workspace=ws, stages=cw.BWD_DQ, stream=s2)
+    torch.cuda.synchronize()
+    assert torch.equal(dq1, dq2) and torch.equal(dk1, dk2) and torch.equal(dv1, dv2)

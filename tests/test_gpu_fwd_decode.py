@@ -180,3 +180,15 @@ def test_decode_128k_config(cuda_device):
     pos[3] = 70000
     pos[5] = 4000
     _check_decode(B, 40, 8, 128, 131072, pat, pos, cuda_device, sample_b=[0, 3, 5, 15], cuda_gen=True)
+
+
+def test_device_wait_timeout_is_reported_and_context_survives(cuda_device):
+    """A device-side wait that runs out sets the workspace status word; the kernel returns, the
+    host reads COWA_ERR_TIMEOUT, and the next call on the same context is correct."""
+    import ctypes
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda_device)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert cw.lib().cowa_debug_wait_timeout(ctypes.c_void_p(ws.data_ptr()), 256, 50_000_000, stream) == 0
+    assert cw.workspace_status(ws) == 6          # COWA_ERR_TIMEOUT, and the word is cleared
+    assert cw.workspace_status(ws) == 0
+    _check_fwd_full(1, 300, 4, 2, 64, cw.Pattern(8, 32, 300, 2), cuda_device, extra=5)
