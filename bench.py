@@ -98,16 +98,19 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def _traffic_record(kernel_file: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+def _traffic_record(kernel: str, kernel_file: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary (profiles/traffic.txt:
+    kernel, source file, sha256 prefix of that file when captured, bytes per launch), or None
+    when the source has changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "structured_sparse_attention_cowa_b200", "csrc", kernel_file)
     try:
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         for line in open(path):
             parts = line.split()
-            if len(parts) >= 3 and parts[0] == kernel_file and parts[1] == sha:
-                return float(parts[2])
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == kernel_file \
+                    and parts[2] == sha:
+                return float(parts[3])
     except Exception:
         pass
     return None
@@ -445,13 +448,13 @@ def run_cowa(args, world, rank, local):
     if bound == "tensor":
         achieved = work / (t_ms * 1e-3) / 1e12
         roofline = {"kernel": top, "bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                    "frac": achieved / sustained, "traffic": _traffic_record(src),
+                    "frac": achieved / sustained, "traffic": _traffic_record(top, src),
                     "peak_source": f"{peak_src} bf16 dense, sustained",
                     "algorithmic": f"{work:.4e} FLOP per launch = {per} x visible pairs ({pairs:.4e})"}
     else:
         achieved = work / (t_ms * 1e-3) / 1e9
         roofline = {"kernel": top, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": _traffic_record(src),
+                    "frac": achieved / hbm, "traffic": _traffic_record(top, src),
                     "peak_source": f"{peak_src} HBM copy",
                     "algorithmic": f"{work:.4e} visible K/V bytes per call"}
     roofline["all_kernels_ms"] = {kname: v[0] for kname, v in kernels.items()}

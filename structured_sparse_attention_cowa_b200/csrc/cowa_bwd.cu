@@ -13,7 +13,9 @@
 //      interval keys are seen by every later query, band keys by the next L queries) for
 //      every query head of the group.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the
 //      elementwise softmax writes P^T and dS^T back into TMEM as bf16, where they are the A
-//      operand of dV += P^T dO and dK += dS^T Q (tcgen05 MMA with A in TMEM);
+//      operand of dV += P^T dO and dK += dS^T Q (tcgen05 MMA with A in TMEM).  The packed
+//      P^T / dS^T sit at columns that overlap only the S^T / dP^T columns the writing warp has
+//      already read (A operands start at column 32 / 160), so no warp waits for another;
 //   3. dQ: one CTA per (b, query head h, 128-row tile i) over the forward tile plan.  The
 //      softmax warps load S and dP of a KV tile into registers and release them at once, so
 //      the MMA warp computes S and dP of the next tile while dS of this one is being formed;
@@ -22,6 +24,8 @@
 // lane quadrant, each owning half of the columns), warp 8 TMA producer, warp 9 MMA issuer.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "cowa_internal.h"
 #include "exp2_poly.cuh"
@@ -55,9 +59,10 @@ struct BwdGeom {
   // dK/dV kernel: K, V resident + 2 slots of {Q, dO, stats}
   static constexpr int kSlotKV = 2 * kTileBytes + kStatBytes;
   static constexpr int kSmemKV = 2 * kTileBytes + 2 * kSlotKV + 1024;
-  // dQ kernel: Q, dO resident + 2 slots of {K, V}
-  static constexpr int kSlotQ = 2 * kTileBytes;
-  static constexpr int kSmemQ = 2 * kTileBytes + 2 * kSlotQ + 1024;
+  // dQ kernel: Q, dO resident + a 3-slot K ring (a K tile lives until its dQ MMA) and a
+  // 2-slot V ring (a V tile is free once its dP MMA is done)
+  static constexpr int kKSlots = 3, kVSlots = 2;
+  static constexpr int kSmemQ = (2 + kKSlots + kVSlots) * kTileBytes + 1024;
   static constexpr int kColAcc = 256;  // first accumulator column
 };
 
@@ -94,20 +99,16 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_consta
   }
 }
 
-// Pack 64 fp32 values (as two 32-column halves) into 32 bf16x2 words.
-__device__ __forceinline__ void pack64(const float* v, uint32_t* w) {
-#pragma unroll
-  for (int c = 0; c < 32; ++c) w[c] = ptx::pack_bf16(v[2 * c], v[2 * c + 1]);
-}
-
 // ------------------------------------------------------------------------------ dK / dV
+// TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [256+D, 256+2D); the packed
+// bf16 P^T and dS^T (64 columns each) start at kColPT / kColDST.
+constexpr uint32_t kColPT = 32, kColDST = 160;
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using Geo = BwdGeom<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full, ld_done, p_ready, acc_full,
-      mma_final;
+  __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full, p_ready, acc_full, mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -131,7 +132,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     ptx::mbar_init(&kv_full, 1);
     for (int s = 0; s < 2; ++s) { ptx::mbar_init(&slot_full[s], 1); ptx::mbar_init(&slot_empty[s], 1); }
     ptx::mbar_init(&sdp_full, 1);
-    ptx::mbar_init(&ld_done, kComputeWarps);
     ptx::mbar_init(&p_ready, kComputeWarps);
     ptx::mbar_init(&acc_full, 1);
     ptx::mbar_init(&mma_final, 1);
@@ -206,11 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + 0 + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + kColPT + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
                            idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, tmem + 128 + kk * 8,
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, tmem + kColDST + kk * 8,
                            ptx::smem_desc_sw128(qa + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
         ptx::mma_commit(&slot_empty[slot]);
       }
@@ -234,46 +234,55 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       const bool need_mask = !tile_full(a.pat, iv, t0, imin(a.N, t0 + kTile), s0, s1);
       if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
-      uint32_t sv[64], pv[64];
-      ptx::tmem_ld32(lane_base + half * 64, sv);
-      ptx::tmem_ld32(lane_base + half * 64 + 32, sv + 32);
-      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);
-      ptx::tmem_ld32(lane_base + 128 + half * 64 + 32, pv + 32);
-      ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&ld_done);
       const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes);
-      // all lanes read the same statistics: 16-byte broadcast loads
-      const float4* lse4 = reinterpret_cast<const float4*>(stat + half * 64);
-      const float4* del4 = reinterpret_cast<const float4*>(stat + 128 + half * 64);
       const bool use_poly = !need_mask && t0 + kTile <= a.N;
-      float pf[64], df[64];
+      // Two chunks of 32 query columns.  Chunk c's packed P^T / dS^T go to columns
+      // kColPT/kColDST + 32*half + 16*c, which overlap only this warp's own S^T / dP^T columns;
+      // half 0 reads its chunk 1 first and half 1 its chunk 0, so nothing is overwritten unread.
+      // the element loop is instantiated with and without the mask, chosen once per tile, so
+      // fully visible tiles carry no per-element mask arithmetic
+      auto chunks = [&](auto masked) {
+        constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 ls = lse4[c4], dl = del4[c4];
-        const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half == 0 ? 1 - cc : cc;
+          const int q0 = half * 64 + c * 32;  // first query column of the chunk
+          uint32_t sv[32], pv[32];
+          ptx::tmem_ld32(lane_base + q0, sv);
+          ptx::tmem_ld32(lane_base + 128 + q0, pv);
+          ptx::tmem_wait_ld();
+          // all lanes read the same statistics: 16-byte broadcast loads
+          const float4* lse4 = reinterpret_cast<const float4*>(stat + q0);
+          const float4* del4 = reinterpret_cast<const float4*>(stat + 128 + q0);
+          uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c4 * 4 + e;
-          const float x = fmaf(__uint_as_float(sv[c]), sl2, -lsv[e]);
-          float p = (use_poly && poly_col<COWA_DKDV_POLY_MASK>(c)) ? exp2_fma(x) : ptx::ex2(x);
-          if (need_mask) {
-            const int t = t0 + half * 64 + c;
-            if (!(t >= s && t < t_hi)) p = 0.f;
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 ls = lse4[c4], dl = del4[c4];
+            const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
+            float pf[4], df[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int cl = c4 * 4 + e;
+              const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lsv[e]);
+              float p = (!kMask && use_poly && poly_col<COWA_DKDV_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
+              if (kMask) {
+                const int t = t0 + q0 + cl;
+                if (!(t >= s && t < t_hi)) p = 0.f;
+              }
+              pf[e] = p;
+              df[e] = p * (__uint_as_float(pv[cl]) - dlv[e]);
+            }
+            pw[2 * c4] = ptx::pack_bf16(pf[0], pf[1]);
+            pw[2 * c4 + 1] = ptx::pack_bf16(pf[2], pf[3]);
+            dw[2 * c4] = ptx::pack_bf16(df[0], df[1]);
+            dw[2 * c4 + 1] = ptx::pack_bf16(df[2], df[3]);
           }
-          pf[c] = p;
-          df[c] = p * (__uint_as_float(pv[c]) - dlv[e]);
+          ptx::tmem_st16(lane_base + kColPT + 32 * half + 16 * c, pw);
+          ptx::tmem_st16(lane_base + kColDST + 32 * half + 16 * c, dw);
         }
-      }
-      uint32_t pw[32], dw[32];
-      pack64(pf, pw);
-      pack64(df, dw);
-      // every compute warp must have read S^T / dP^T before P^T / dS^T overwrite them
-      if (!(ok = ptx::mbar_wait_warp(&ld_done, n & 1, &abort_flag, a.status))) break;
-      ptx::tc_fence_after();
-      ptx::tmem_st32(lane_base + half * 32, pw);
-      ptx::tmem_st32(lane_base + 128 + half * 32, dw);
+      };
+      if (need_mask) chunks(std::true_type{});
+      else chunks(std::false_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -327,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   // ds_ready is per dS buffer: a barrier can then never run two phases ahead of its waiter
-  __shared__ __align__(8) uint64_t q_full, kv_full[2], kv_empty[2], sdp_full, consumed, ds_ready[2], acc_full,
-      mma_final;
+  __shared__ __align__(8) uint64_t q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, consumed,
+      ds_ready[2], acc_full, mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -344,14 +353,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   const Range iv = interval_of(a.pat, g);
   const Tiles T = plan_tiles(a.pat, iv, t0, t1);
   const int ntiles = T.count;
+  constexpr int KS = Geo::kKSlots, VS = Geo::kVSlots;
 
   uint8_t* sQ = smem;
   uint8_t* sDO = smem + Geo::kTileBytes;
-  uint8_t* sSlot = smem + 2 * Geo::kTileBytes;
+  uint8_t* sK = smem + 2 * Geo::kTileBytes;
+  uint8_t* sV = sK + KS * Geo::kTileBytes;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 1);
-    for (int s = 0; s < 2; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < KS; ++s) { ptx::mbar_init(&k_full[s], 1); ptx::mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < VS; ++s) { ptx::mbar_init(&v_full[s], 1); ptx::mbar_init(&v_empty[s], 1); }
     ptx::mbar_init(&sdp_full, 1);
     ptx::mbar_init(&consumed, kComputeWarps);
     ptx::mbar_init(&ds_ready[0], kComputeWarps);
@@ -383,28 +395,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       cur.init(T);
       int issued = 0;
       for (int n = 0; n < ntiles; ++n, cur.next(T)) {
-        const int slot = n & 1;
-        if (n >= 2 && !ptx::mbar_wait(&kv_empty[slot], ((n >> 1) - 1) & 1, &abort_flag, a.status)) break;
-        uint8_t* dst = sSlot + slot * Geo::kSlotQ;
-        ptx::mbar_arrive_expect_tx(&kv_full[slot], Geo::kSlotQ);
-        for (int u = 0; u < D / 64; ++u) {
-          ptx::tma_load_4d(dst + u * 16384, &a.tm_k, &kv_full[slot], u * 64, cur.j * kTile, g, b);
-          ptx::tma_load_4d(dst + Geo::kTileBytes + u * 16384, &a.tm_v, &kv_full[slot], u * 64, cur.j * kTile, g, b);
+        const int ks = n % KS, vs = n % VS;
+        if (n >= KS && !ptx::mbar_wait(&k_empty[ks], ((n / KS) - 1) & 1, &abort_flag, a.status)) break;
+        ptx::mbar_arrive_expect_tx(&k_full[ks], Geo::kTileBytes);
+        for (int u = 0; u < D / 64; ++u)
+          ptx::tma_load_4d(sK + ks * Geo::kTileBytes + u * 16384, &a.tm_k, &k_full[ks], u * 64, cur.j * kTile, g, b);
+        if (n >= VS && !ptx::mbar_wait(&v_empty[vs], ((n / VS) - 1) & 1, &abort_flag, a.status)) {
+          issued = -(n + 1);  // K of tile n is in flight, V is not
+          break;
         }
+        ptx::mbar_arrive_expect_tx(&v_full[vs], Geo::kTileBytes);
+        for (int u = 0; u < D / 64; ++u)
+          ptx::tma_load_4d(sV + vs * Geo::kTileBytes + u * 16384, &a.tm_v, &v_full[vs], u * 64, cur.j * kTile, g, b);
         issued = n + 1;
       }
+      // drain: every copy issued must have landed before the CTA exits
       ptx::mbar_wait(&q_full, 0, nullptr, a.status);
-      for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
-        ptx::mbar_wait(&kv_full[n & 1], (n >> 1) & 1, nullptr, a.status);
+      const int nk = issued < 0 ? -issued : issued, nv = issued < 0 ? -issued - 1 : issued;
+      for (int n = (nk > KS ? nk - KS : 0); n < nk; ++n) ptx::mbar_wait(&k_full[n % KS], (n / KS) & 1, nullptr, a.status);
+      for (int n = (nv > VS ? nv - VS : 0); n < nv; ++n) ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, nullptr, a.status);
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ), do_addr = ptx::smem_u32(sDO), slot_addr = ptx::smem_u32(sSlot);
-      // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns
-      auto issue_sdp = [&](int n) {
-        const uint32_t ka = slot_addr + (n & 1) * Geo::kSlotQ, va = ka + Geo::kTileBytes;
+      const uint32_t q_addr = ptx::smem_u32(sQ), do_addr = ptx::smem_u32(sDO);
+      const uint32_t k_addr = ptx::smem_u32(sK), v_addr = ptx::smem_u32(sV);
+      // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns; V_n is free afterwards
+      auto issue_sdp = [&](int n) -> bool {
+        if (!ptx::mbar_wait(&k_full[n % KS], (n / KS) & 1, &abort_flag, a.status)) return false;
+        if (!ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, &abort_flag, a.status)) return false;
+        ptx::tc_fence_after();
+        const uint32_t ka = k_addr + (n % KS) * Geo::kTileBytes, va = v_addr + (n % VS) * Geo::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -418,31 +440,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
                            ptx::smem_desc_sw128(va + off, 16, 1024), idesc_s, kk > 0);
         }
         ptx::mma_commit(&sdp_full);
+        ptx::mma_commit(&v_empty[n % VS]);
+        return true;
       };
       bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
       ptx::tc_fence_after();
-      if (ok && ntiles > 0 && (ok = ptx::mbar_wait(&kv_full[0], 0, &abort_flag, a.status))) {
-        ptx::tc_fence_after();
-        issue_sdp(0);
-      }
+      if (ok && ntiles > 0) ok = issue_sdp(0);
       for (int n = 0; ok && n < ntiles; ++n) {
         // the softmax holds S(n), dP(n) in registers: compute the next tile's S and dP now
         if (!(ok = ptx::mbar_wait(&consumed, n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
-        if (n + 1 < ntiles) {
-          if (!(ok = ptx::mbar_wait(&kv_full[(n + 1) & 1], ((n + 1) >> 1) & 1, &abort_flag, a.status))) break;
-          ptx::tc_fence_after();
-          issue_sdp(n + 1);
-        }
+        if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
         if (!(ok = ptx::mbar_wait(&ds_ready[n & 1], (n >> 1) & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
         // dQ += dS K : A = dS (TMEM buffer n & 1), B = K MN-major in smem
-        const uint32_t ka = slot_addr + (n & 1) * Geo::kSlotQ;
+        const uint32_t ka = k_addr + (n % KS) * Geo::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + kColDS + (n & 1) * 64 + kk * 8,
                            ptx::smem_desc_sw128(ka + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(&kv_empty[n & 1]);
+        ptx::mma_commit(&k_empty[n % KS]);
       }
       if (ok) ptx::mma_commit(&acc_full);
       ptx::mma_commit(&mma_final);
@@ -478,26 +495,35 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&consumed);  // S / dP columns may be overwritten now
       const bool use_poly = !need_mask && t < a.N;
-      uint32_t dw[32];
+      // dS buffer n & 1 was last read by dQ(n-2), which the commit of S(n) covers.  The element
+      // loop is instantiated with and without the mask, chosen once per tile.
+      auto chunks = [&](auto masked) {
+        constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        float d2[2];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dw[16];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * c2 + e;
-          const float x = fmaf(__uint_as_float(sv[c]), sl2, -lse2);
-          float p = (use_poly && poly_col<COWA_DQ_POLY_MASK>(c)) ? exp2_fma(x) : ptx::ex2(x);
-          if (need_mask) {
-            const int s = s0 + half * 64 + c;
-            const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
-            if (!vis) p = 0.f;
+          for (int c2 = 0; c2 < 16; ++c2) {
+            float d2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int cl = 32 * c + 2 * c2 + e;
+              const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lse2);
+              float p = (!kMask && use_poly && poly_col<COWA_DQ_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
+              if (kMask) {
+                const int s = s0 + half * 64 + cl;
+                const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
+                if (!vis) p = 0.f;
+              }
+              d2[e] = p * (__uint_as_float(pv[cl]) - delta);
+            }
+            dw[c2] = ptx::pack_bf16(d2[0], d2[1]);
           }
-          d2[e] = p * (__uint_as_float(pv[c]) - delta);
+          ptx::tmem_st16(lane_base + kColDS + (n & 1) * 64 + half * 32 + 16 * c, dw);
         }
-        dw[c2] = ptx::pack_bf16(d2[0], d2[1]);
-      }
-      // dS buffer n & 1 was last read by dQ(n-2), which the commit of S(n) covers
-      ptx::tmem_st32(lane_base + kColDS + (n & 1) * 64 + half * 32, dw);
+      };
+      if (need_mask) chunks(std::true_type{});
+      else chunks(std::false_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();

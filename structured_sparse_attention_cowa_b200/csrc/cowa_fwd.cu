@@ -268,9 +268,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
             if (!vis) xr[c] = 0xff800000u;  // -inf
           }
         }
-        float mx = -INFINITY;
+        // row max as a shallow tree (8 independent partial maxima), not a 64-deep chain
+        float pm[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) mx = ptx::fmax3(mx, __uint_as_float(xr[c]), __uint_as_float(xr[c + 1]));
+        for (int e = 0; e < 8; ++e) pm[e] = fmaxf(__uint_as_float(xr[e]), __uint_as_float(xr[e + 8]));
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pm[e] = ptx::fmax3(pm[e], __uint_as_float(xr[c + e]), __uint_as_float(xr[c + 8 + e]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
         const float m_new = fmaxf(m_used, mx * sl2);
         // lazy rescale: only when the running max grows by more than 2^8 (or first finite max);
         // PV_k(n-1) has completed (the commit of S_k(n) covers it), so O_k is stable here
@@ -295,6 +301,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         }
         const float m_eff = m_used == -INFINITY ? 0.f : m_used;
         const uint64_t negm = ptx::f2_pack(-m_eff, -m_eff);
+        uint64_t ts[4];  // this tile's row sum, 4 independent packed accumulators
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ts[e] = ptx::f2_pack(0.f, 0.f);
         // P = 2^(s*scale*log2e - m), rounded to bf16, back into TMEM over the S columns
         // (masked scores are -inf and give exactly 0)
 #pragma unroll
@@ -314,11 +323,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
               p0 = poly_col(c) ? exp2_fma(e0) : ptx::ex2(e0);
               p1 = poly_col(c + 1) ? exp2_fma(e1) : ptx::ex2(e1);
             }
-            lsum = ptx::f2_add(lsum, ptx::f2_pack(p0, p1));
+            ts[c2 & 3] = ptx::f2_add(ts[c2 & 3], ptx::f2_pack(p0, p1));
             pw[c2] = ptx::pack_bf16(p0, p1);
           }
           ptx::tmem_st32(s_tm + 32 * h, pw);
         }
+        lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ts[0], ts[1]), ptx::f2_add(ts[2], ts[3])));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
