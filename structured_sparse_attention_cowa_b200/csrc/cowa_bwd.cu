@@ -11,11 +11,13 @@
 //   2. dK/dV: one CTA per (b, KV head g, 128-key tile j); K_j, V_j stay in shared memory and
 //      the CTA walks the single contiguous range of query tiles that see tile j (sink and
 //      interval keys are seen by every later query, band keys by the next L queries) for
-//      every query head of the group.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the
-//      elementwise softmax writes P^T and dS^T back into TMEM as bf16, where they are the A
-//      operand of dV += P^T dO and dK += dS^T Q (tcgen05 MMA with A in TMEM).  The packed
-//      P^T / dS^T sit at columns that overlap only the S^T / dP^T columns the writing warp has
-//      already read (A operands start at column 32 / 160), so no warp waits for another;
+//      every query head of the group, in sub-steps of 64 query rows.  S^T = K Q^T and
+//      dP^T = V dO^T of a sub-step land in one of two TMEM buffers, so the MMAs of sub-step
+//      m+1 run while the elementwise softmax works on sub-step m; the softmax writes P^T and
+//      dS^T back into the buffer as bf16, where they are the A operand of dV += P^T dO and
+//      dK += dS^T Q (tcgen05 MMA with A in TMEM).  The packed P^T / dS^T sit at columns that
+//      overlap only the S^T / dP^T columns the writing warp has already read, so no warp
+//      waits for another;
 //   3. dQ: one CTA per (b, query head h, 128-row tile i) over the forward tile plan.  The
 //      softmax warps load S and dP of a KV tile into registers and release them at once, so
 //      the MMA warp computes S and dP of the next tile while dS of this one is being formed;
@@ -100,15 +102,18 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------------------------ dK / dV
-// TMEM columns: S^T [0,128), dP^T [128,256), dV [256, 256+D), dK [256+D, 256+2D); the packed
-// bf16 P^T and dS^T (64 columns each) start at kColPT / kColDST.
-constexpr uint32_t kColPT = 32, kColDST = 160;
+// TMEM columns: two sub-step buffers at 0 and 128, each S^T [+0, +64) and dP^T [+64, +128)
+// for 64 query rows; dV [256, 256+D), dK [256+D, 256+2D).  The packed bf16 P^T and dS^T of a
+// buffer (32 columns each) start at +kColPT / +kColDST.
+constexpr uint32_t kColPT = 16, kColDST = 80;
+constexpr int kSub = 64;  // query rows per sub-step
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using Geo = BwdGeom<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full, p_ready, acc_full, mma_final;
+  __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full[2], p_ready[2], acc_full,
+      mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -131,8 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
   if (threadIdx.x == 0) {
     ptx::mbar_init(&kv_full, 1);
     for (int s = 0; s < 2; ++s) { ptx::mbar_init(&slot_full[s], 1); ptx::mbar_init(&slot_empty[s], 1); }
-    ptx::mbar_init(&sdp_full, 1);
-    ptx::mbar_init(&p_ready, kComputeWarps);
+    for (int bb = 0; bb < 2; ++bb) {
+      ptx::mbar_init(&sdp_full[bb], 1);
+      ptx::mbar_init(&p_ready[bb], kComputeWarps);
+    }
     ptx::mbar_init(&acc_full, 1);
     ptx::mbar_init(&mma_final, 1);
     abort_flag = 0;
@@ -146,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  const int nsub = 2 * nsteps;  // 64-row sub-steps
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -178,41 +186,52 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, kSub, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
       const uint32_t k_addr = ptx::smem_u32(sK), v_addr = ptx::smem_u32(sV), slot_addr = ptx::smem_u32(sSlot);
-      bool ok = ptx::mbar_wait(&kv_full, 0, &abort_flag, a.status);
-      ptx::tc_fence_after();
-      for (int n = 0; ok && n < nsteps; ++n) {
-        const int slot = n & 1;
-        const uint32_t qa = slot_addr + slot * Geo::kSlotKV, da = qa + Geo::kTileBytes;
-        if (!(ok = ptx::mbar_wait(&slot_full[slot], (n >> 1) & 1, &abort_flag, a.status))) break;
+      // S^T, dP^T of sub-step m (query rows 64*(m&1).. of step m>>1) into buffer m & 1.  The
+      // buffer's previous P^T / dS^T were read by dV / dK of sub-step m-2, issued earlier.
+      auto issue_sdp = [&](int m) -> bool {
+        const int n = m >> 1, hq = m & 1;
+        if (hq == 0 && !ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, &abort_flag, a.status)) return false;
         ptx::tc_fence_after();
+        const uint32_t qa = slot_addr + (n & 1) * Geo::kSlotKV + hq * (kSub * 128), da = qa + Geo::kTileBytes;
+        const uint32_t buf = tmem + 128 * (m & 1);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + 0, ptx::smem_desc_sw128(k_addr + off, 16, 1024),
+          ptx::mma_bf16_ss(buf, ptx::smem_desc_sw128(k_addr + off, 16, 1024),
                            ptx::smem_desc_sw128(qa + off, 16, 1024), idesc_s, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + 128, ptx::smem_desc_sw128(v_addr + off, 16, 1024),
+          ptx::mma_bf16_ss(buf + 64, ptx::smem_desc_sw128(v_addr + off, 16, 1024),
                            ptx::smem_desc_sw128(da + off, 16, 1024), idesc_s, kk > 0);
         }
-        ptx::mma_commit(&sdp_full);
-        if (!(ok = ptx::mbar_wait(&p_ready, n & 1, &abort_flag, a.status))) break;
+        ptx::mma_commit(&sdp_full[m & 1]);
+        return true;
+      };
+      bool ok = ptx::mbar_wait(&kv_full, 0, &abort_flag, a.status);
+      ptx::tc_fence_after();
+      if (ok && nsub > 0) ok = issue_sdp(0);
+      for (int m = 0; ok && m < nsub; ++m) {
+        if (m + 1 < nsub && !(ok = issue_sdp(m + 1))) break;
+        if (!(ok = ptx::mbar_wait(&p_ready[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
+        const int n = m >> 1, hq = m & 1;
+        const uint32_t qa = slot_addr + (n & 1) * Geo::kSlotKV + hq * (kSub * 128), da = qa + Geo::kTileBytes;
+        const uint32_t buf = tmem + 128 * (m & 1);
         // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + kColPT + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
-                           idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc, buf + kColPT + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
+                           idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, tmem + kColDST + kk * 8,
-                           ptx::smem_desc_sw128(qa + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(&slot_empty[slot]);
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, buf + kColDST + kk * 8,
+                           ptx::smem_desc_sw128(qa + kk * 2048, 16384, 1024), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
+        if (hq == 1) ptx::mma_commit(&slot_empty[n & 1]);
       }
       if (ok) ptx::mma_commit(&acc_full);
       ptx::mma_commit(&mma_final);
@@ -228,65 +247,59 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     const int t_hi = special ? a.N : imin(a.N, s + a.pat.L);  // rows [s, t_hi) see key s
     const float sl2 = a.scale_log2;
     bool ok = true;
-    for (int n = 0; n < nsteps; ++n) {
-      const int i = i_lo + n / grp;
-      const int t0 = i * kTile;
-      const bool need_mask = !tile_full(a.pat, iv, t0, imin(a.N, t0 + kTile), s0, s1);
-      if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
+    for (int m = 0; m < nsub; ++m) {
+      const int n = m >> 1, hq = m & 1;
+      const int t0 = (i_lo + n / grp) * kTile + hq * kSub;  // first query row of the sub-step
+      const bool need_mask = !tile_full(a.pat, iv, t0, imin(a.N, t0 + kSub), s0, s1);
+      if (!(ok = ptx::mbar_wait_warp(&sdp_full[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
-      const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes);
-      const bool use_poly = !need_mask && t0 + kTile <= a.N;
-      // Two chunks of 32 query columns.  Chunk c's packed P^T / dS^T go to columns
-      // kColPT/kColDST + 32*half + 16*c, which overlap only this warp's own S^T / dP^T columns;
-      // half 0 reads its chunk 1 first and half 1 its chunk 0, so nothing is overwritten unread.
-      // the element loop is instantiated with and without the mask, chosen once per tile, so
-      // fully visible tiles carry no per-element mask arithmetic
-      auto chunks = [&](auto masked) {
+      const uint32_t buf = lane_base + 128 * (m & 1);
+      // this warp's 32 query columns of the sub-step
+      uint32_t sv[32], pv[32];
+      ptx::tmem_ld32(buf + 32 * half, sv);
+      ptx::tmem_ld32(buf + 64 + 32 * half, pv);
+      ptx::tmem_wait_ld();
+      const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes) +
+                          hq * kSub + 32 * half;
+      const bool use_poly = !need_mask && t0 + kSub <= a.N;
+      // the element loop is instantiated with and without the mask, chosen once per sub-step
+      auto body = [&](auto masked) {
         constexpr bool kMask = decltype(masked)::value;
+        const float4* lse4 = reinterpret_cast<const float4*>(stat);
+        const float4* del4 = reinterpret_cast<const float4*>(stat + 128);
+        uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half == 0 ? 1 - cc : cc;
-          const int q0 = half * 64 + c * 32;  // first query column of the chunk
-          uint32_t sv[32], pv[32];
-          ptx::tmem_ld32(lane_base + q0, sv);
-          ptx::tmem_ld32(lane_base + 128 + q0, pv);
-          ptx::tmem_wait_ld();
-          // all lanes read the same statistics: 16-byte broadcast loads
-          const float4* lse4 = reinterpret_cast<const float4*>(stat + q0);
-          const float4* del4 = reinterpret_cast<const float4*>(stat + 128 + q0);
-          uint32_t pw[16], dw[16];
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 ls = lse4[c4], dl = del4[c4];
+          const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
+          float pf[4], df[4];
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4) {
-            const float4 ls = lse4[c4], dl = del4[c4];
-            const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
-            float pf[4], df[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int cl = c4 * 4 + e;
-              const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lsv[e]);
-              float p = (!kMask && use_poly && poly_col<COWA_DKDV_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
-              if (kMask) {
-                const int t = t0 + q0 + cl;
-                if (!(t >= s && t < t_hi)) p = 0.f;
-              }
-              pf[e] = p;
-              df[e] = p * (__uint_as_float(pv[cl]) - dlv[e]);
+          for (int e = 0; e < 4; ++e) {
+            const int cl = c4 * 4 + e;
+            const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lsv[e]);
+            float p = (!kMask && use_poly && poly_col<COWA_DKDV_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
+            if (kMask) {
+              const int t = t0 + 32 * half + cl;
+              if (!(t >= s && t < t_hi)) p = 0.f;
             }
-            pw[2 * c4] = ptx::pack_bf16(pf[0], pf[1]);
-            pw[2 * c4 + 1] = ptx::pack_bf16(pf[2], pf[3]);
-            dw[2 * c4] = ptx::pack_bf16(df[0], df[1]);
-            dw[2 * c4 + 1] = ptx::pack_bf16(df[2], df[3]);
+            pf[e] = p;
+            df[e] = p * (__uint_as_float(pv[cl]) - dlv[e]);
           }
-          ptx::tmem_st16(lane_base + kColPT + 32 * half + 16 * c, pw);
-          ptx::tmem_st16(lane_base + kColDST + 32 * half + 16 * c, dw);
+          pw[2 * c4] = ptx::pack_bf16(pf[0], pf[1]);
+          pw[2 * c4 + 1] = ptx::pack_bf16(pf[2], pf[3]);
+          dw[2 * c4] = ptx::pack_bf16(df[0], df[1]);
+          dw[2 * c4 + 1] = ptx::pack_bf16(df[2], df[3]);
         }
+        // packed columns of this warp's 32 query columns lie inside the columns it just read
+        ptx::tmem_st16(buf + kColPT + 16 * half, pw);
+        ptx::tmem_st16(buf + kColDST + 16 * half, dw);
       };
-      if (need_mask) chunks(std::true_type{});
-      else chunks(std::false_type{});
+      if (need_mask) body(std::true_type{});
+      else body(std::false_type{});
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&p_ready);
+      if (lane == 0) ptx::mbar_arrive(&p_ready[m & 1]);
     }
     if (ok && nsteps > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
       ptx::tc_fence_after();

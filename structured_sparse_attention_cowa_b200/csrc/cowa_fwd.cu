@@ -35,6 +35,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "cowa_internal.h"
 #include "exp2_poly.cuh"
 #include "kernel_common.cuh"
@@ -305,29 +307,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 4; ++e) ts[e] = ptx::f2_pack(0.f, 0.f);
         // P = 2^(s*scale*log2e - m), rounded to bf16, back into TMEM over the S columns
-        // (masked scores are -inf and give exactly 0)
+        // (masked scores are -inf and give exactly 0).  Two instantiations so that the
+        // FMA-pipe share (unmasked tiles only) is decided at compile time per loop.
+        auto exp_tile = [&](auto fma_share) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pw[32];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pw[32];
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const int c = 64 * h + 2 * c2;
-            float e0, e1;
-            ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), sl2x2, negm),
-                           e0, e1);
-            float p0, p1;
-            if (need_mask) {
-              p0 = ptx::ex2(e0);
-              p1 = ptx::ex2(e1);
-            } else {
-              p0 = poly_col(c) ? exp2_fma(e0) : ptx::ex2(e0);
-              p1 = poly_col(c + 1) ? exp2_fma(e1) : ptx::ex2(e1);
+            for (int c2 = 0; c2 < 32; ++c2) {
+              const int c = 64 * h + 2 * c2;
+              float e0, e1;
+              ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), sl2x2, negm),
+                             e0, e1);
+              float p0, p1;
+              if (decltype(fma_share)::value && poly_col(c) && poly_col(c + 1)) {
+                exp2_fma_x2(e0, e1, p0, p1);  // a pair on the FMA pipe
+              } else {
+                p0 = (decltype(fma_share)::value && poly_col(c)) ? exp2_fma(e0) : ptx::ex2(e0);
+                p1 = (decltype(fma_share)::value && poly_col(c + 1)) ? exp2_fma(e1) : ptx::ex2(e1);
+              }
+              ts[c2 & 3] = ptx::f2_add(ts[c2 & 3], ptx::f2_pack(p0, p1));
+              pw[c2] = ptx::pack_bf16(p0, p1);
             }
-            ts[c2 & 3] = ptx::f2_add(ts[c2 & 3], ptx::f2_pack(p0, p1));
-            pw[c2] = ptx::pack_bf16(p0, p1);
+            ptx::tmem_st32(s_tm + 32 * h, pw);
           }
-          ptx::tmem_st32(s_tm + 32 * h, pw);
-        }
+        };
+        if (COWA_FWD_POLY_MASK == 0 || need_mask)
+          exp_tile(std::false_type{});
+        else
+          exp_tile(std::true_type{});
         lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ts[0], ts[1]), ptx::f2_add(ts[2], ts[3])));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();

@@ -37,4 +37,31 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + e);
 }
 
+// Two values at once with packed fp32x2 arithmetic (same method and constants as above);
+// 7 instructions per element instead of 10.  lo/hi in the low/high word of each operand.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -120.0f);
+  x1 = fmaxf(x1, -120.0f);
+  uint64_t xx, t, mg, n, f, p;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(mg) : "f"(kMagic));
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xx), "l"(mg));   // magic + floor(x)
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(mg));       // floor(x)
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(f) : "l"(xx), "l"(n));       // x - floor(x) in [0, 1)
+  uint64_t c3, c2, c1, c0;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(kExp2C3));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(kExp2C2));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(kExp2C1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(kExp2C0));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+  float t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(p0), "=f"(p1) : "l"(p));
+  y0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - __float_as_int(kMagic)) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - __float_as_int(kMagic)) << 23));
+}
+
 }  // namespace cowa

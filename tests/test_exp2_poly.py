@@ -36,3 +36,12 @@ def test_float32_evaluation_error_bound():
     # clamped below -120: a tiny positive normal float, never negative, denormal or NaN
     y = exp2_poly_fit.eval_f32(c32, np.array([-1000.0, -121.0], np.float32))
     assert (y > np.float32(2.0 ** -121)).all() and (y < np.float32(2.0 ** -119)).all()
+
+
+def test_packed_variant_uses_the_same_steps():
+    """The packed device variant repeats the scalar steps on pairs; its header text must carry
+    the same constants and clamp (one source of truth: the kExp2C* constants)."""
+    txt = open(os.path.join(CSRC, "exp2_poly.cuh")).read()
+    body = txt[txt.index("exp2_fma_x2"):]
+    for name in ("kExp2C3", "kExp2C2", "kExp2C1", "kExp2C0", "-120.0f", "12582912.0f"):
+        assert name in body
