@@ -185,58 +185,61 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
         ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, nullptr, a.status);
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, kSub, false, false);
-      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
-      const uint32_t k_addr = ptx::smem_u32(sK), v_addr = ptx::smem_u32(sV), slot_addr = ptx::smem_u32(sSlot);
-      // S^T, dP^T of sub-step m (query rows 64*(m&1).. of step m>>1) into buffer m & 1.  The
-      // buffer's previous P^T / dS^T were read by dV / dK of sub-step m-2, issued earlier.
-      auto issue_sdp = [&](int m) -> bool {
-        const int n = m >> 1, hq = m & 1;
-        if (hq == 0 && !ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, &abort_flag, a.status)) return false;
-        ptx::tc_fence_after();
-        const uint32_t qa = slot_addr + (n & 1) * Geo::kSlotKV + hq * (kSub * 128), da = qa + Geo::kTileBytes;
-        const uint32_t buf = tmem + 128 * (m & 1);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(buf, ptx::smem_desc_sw128(k_addr + off, 16, 1024),
-                           ptx::smem_desc_sw128(qa + off, 16, 1024), idesc_s, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(buf + 64, ptx::smem_desc_sw128(v_addr + off, 16, 1024),
-                           ptx::smem_desc_sw128(da + off, 16, 1024), idesc_s, kk > 0);
-        }
-        ptx::mma_commit(&sdp_full[m & 1]);
-        return true;
-      };
-      bool ok = ptx::mbar_wait(&kv_full, 0, &abort_flag, a.status);
+    // whole warp on the issue path, one elected lane issues (uniform descriptors)
+    constexpr uint32_t idesc_s = ptx::idesc_bf16(128, kSub, false, false);
+    constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+    const uint64_t k_desc = ptx::smem_desc_sw128(ptx::smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = ptx::smem_desc_sw128(ptx::smem_u32(sV), 16, 1024);
+    const uint64_t slot_desc_k = ptx::smem_desc_sw128(ptx::smem_u32(sSlot), 16, 1024);     // K-major reads
+    const uint64_t slot_desc_mn = ptx::smem_desc_sw128(ptx::smem_u32(sSlot), 16384, 1024);  // MN-major reads
+    // S^T, dP^T of sub-step m (query rows 64*(m&1).. of step m>>1) into buffer m & 1.  The
+    // buffer's previous P^T / dS^T were read by dV / dK of sub-step m-2, issued earlier.
+    auto issue_sdp = [&](int m) -> bool {
+      const int n = m >> 1, hq = m & 1;
+      if (hq == 0 && !ptx::mbar_wait_warp(&slot_full[n & 1], (n >> 1) & 1, &abort_flag, a.status)) return false;
       ptx::tc_fence_after();
-      if (ok && nsub > 0) ok = issue_sdp(0);
-      for (int m = 0; ok && m < nsub; ++m) {
-        if (m + 1 < nsub && !(ok = issue_sdp(m + 1))) break;
-        if (!(ok = ptx::mbar_wait(&p_ready[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        const int n = m >> 1, hq = m & 1;
-        const uint32_t qa = slot_addr + (n & 1) * Geo::kSlotKV + hq * (kSub * 128), da = qa + Geo::kTileBytes;
-        const uint32_t buf = tmem + 128 * (m & 1);
-        // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
+      const uint32_t q_off = (n & 1) * Geo::kSlotKV + hq * (kSub * 128), do_off = q_off + Geo::kTileBytes;
+      const uint32_t buf = tmem + 128 * (m & 1);
 #pragma unroll
-        for (int kk = 0; kk < kSub / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc, buf + kColPT + kk * 8, ptx::smem_desc_sw128(da + kk * 2048, 16384, 1024),
-                           idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < kSub / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc + D, buf + kColDST + kk * 8,
-                           ptx::smem_desc_sw128(qa + kk * 2048, 16384, 1024), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
-        if (hq == 1) ptx::mma_commit(&slot_empty[n & 1]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        ptx::mma_bf16_ss_warp(buf, ptx::desc_advance(k_desc, off), ptx::desc_advance(slot_desc_k, q_off + off),
+                              idesc_s, kk > 0);
       }
-      if (ok) ptx::mma_commit(&acc_full);
-      ptx::mma_commit(&mma_final);
-      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        ptx::mma_bf16_ss_warp(buf + 64, ptx::desc_advance(v_desc, off), ptx::desc_advance(slot_desc_k, do_off + off),
+                              idesc_s, kk > 0);
+      }
+      ptx::mma_commit_warp(&sdp_full[m & 1]);
+      return true;
+    };
+    bool ok = ptx::mbar_wait_warp(&kv_full, 0, &abort_flag, a.status);
+    ptx::tc_fence_after();
+    if (ok && nsub > 0) ok = issue_sdp(0);
+    for (int m = 0; ok && m < nsub; ++m) {
+      if (m + 1 < nsub && !(ok = issue_sdp(m + 1))) break;
+      if (!(ok = ptx::mbar_wait_warp(&p_ready[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      const int n = m >> 1, hq = m & 1;
+      const uint32_t q_off = (n & 1) * Geo::kSlotKV + hq * (kSub * 128), do_off = q_off + Geo::kTileBytes;
+      const uint32_t buf = tmem + 128 * (m & 1);
+      // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
+#pragma unroll
+      for (int kk = 0; kk < kSub / 16; ++kk)
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc, buf + kColPT + kk * 8,
+                              ptx::desc_advance(slot_desc_mn, do_off + kk * 2048), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+      for (int kk = 0; kk < kSub / 16; ++kk)
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc + D, buf + kColDST + kk * 8,
+                              ptx::desc_advance(slot_desc_mn, q_off + kk * 2048), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
+      if (hq == 1) ptx::mma_commit_warp(&slot_empty[n & 1]);
     }
+    if (ok) ptx::mma_commit_warp(&acc_full);
+    ptx::mma_commit_warp(&mma_final);
+    ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise softmax (8 warps)
     const int quad = warp & 3, half = warp >> 2;
@@ -429,55 +432,57 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       for (int n = (nv > VS ? nv - VS : 0); n < nv; ++n) ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, nullptr, a.status);
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ), do_addr = ptx::smem_u32(sDO);
-      const uint32_t k_addr = ptx::smem_u32(sK), v_addr = ptx::smem_u32(sV);
-      // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns; V_n is free afterwards
-      auto issue_sdp = [&](int n) -> bool {
-        if (!ptx::mbar_wait(&k_full[n % KS], (n / KS) & 1, &abort_flag, a.status)) return false;
-        if (!ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, &abort_flag, a.status)) return false;
-        ptx::tc_fence_after();
-        const uint32_t ka = k_addr + (n % KS) * Geo::kTileBytes, va = v_addr + (n % VS) * Geo::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + 0, ptx::smem_desc_sw128(q_addr + off, 16, 1024),
-                           ptx::smem_desc_sw128(ka + off, 16, 1024), idesc_s, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + 128, ptx::smem_desc_sw128(do_addr + off, 16, 1024),
-                           ptx::smem_desc_sw128(va + off, 16, 1024), idesc_s, kk > 0);
-        }
-        ptx::mma_commit(&sdp_full);
-        ptx::mma_commit(&v_empty[n % VS]);
-        return true;
-      };
-      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
+    // whole warp on the issue path, one elected lane issues (uniform descriptors)
+    constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+    const uint64_t q_desc = ptx::smem_desc_sw128(ptx::smem_u32(sQ), 16, 1024);
+    const uint64_t do_desc = ptx::smem_desc_sw128(ptx::smem_u32(sDO), 16, 1024);
+    const uint64_t k_desc = ptx::smem_desc_sw128(ptx::smem_u32(sK), 16, 1024);
+    const uint64_t k_desc_mn = ptx::smem_desc_sw128(ptx::smem_u32(sK), 16384, 1024);
+    const uint64_t v_desc = ptx::smem_desc_sw128(ptx::smem_u32(sV), 16, 1024);
+    // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns; V_n is free afterwards
+    auto issue_sdp = [&](int n) -> bool {
+      if (!ptx::mbar_wait_warp(&k_full[n % KS], (n / KS) & 1, &abort_flag, a.status)) return false;
+      if (!ptx::mbar_wait_warp(&v_full[n % VS], (n / VS) & 1, &abort_flag, a.status)) return false;
       ptx::tc_fence_after();
-      if (ok && ntiles > 0) ok = issue_sdp(0);
-      for (int n = 0; ok && n < ntiles; ++n) {
-        // the softmax holds S(n), dP(n) in registers: compute the next tile's S and dP now
-        if (!(ok = ptx::mbar_wait(&consumed, n & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
-        if (!(ok = ptx::mbar_wait(&ds_ready[n & 1], (n >> 1) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        // dQ += dS K : A = dS (TMEM buffer n & 1), B = K MN-major in smem
-        const uint32_t ka = k_addr + (n % KS) * Geo::kTileBytes;
+      const uint64_t kd = ptx::desc_advance(k_desc, (n % KS) * Geo::kTileBytes);
+      const uint64_t vd = ptx::desc_advance(v_desc, (n % VS) * Geo::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColAcc, tmem + kColDS + (n & 1) * 64 + kk * 8,
-                           ptx::smem_desc_sw128(ka + kk * 2048, 16384, 1024), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(&k_empty[n % KS]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        ptx::mma_bf16_ss_warp(tmem + 0, ptx::desc_advance(q_desc, off), ptx::desc_advance(kd, off), idesc_s, kk > 0);
       }
-      if (ok) ptx::mma_commit(&acc_full);
-      ptx::mma_commit(&mma_final);
-      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        ptx::mma_bf16_ss_warp(tmem + 128, ptx::desc_advance(do_desc, off), ptx::desc_advance(vd, off), idesc_s, kk > 0);
+      }
+      ptx::mma_commit_warp(&sdp_full);
+      ptx::mma_commit_warp(&v_empty[n % VS]);
+      return true;
+    };
+    bool ok = ptx::mbar_wait_warp(&q_full, 0, &abort_flag, a.status);
+    ptx::tc_fence_after();
+    if (ok && ntiles > 0) ok = issue_sdp(0);
+    for (int n = 0; ok && n < ntiles; ++n) {
+      // the softmax holds S(n), dP(n) in registers: compute the next tile's S and dP now
+      if (!(ok = ptx::mbar_wait_warp(&consumed, n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
+      if (!(ok = ptx::mbar_wait_warp(&ds_ready[n & 1], (n >> 1) & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      // dQ += dS K : A = dS (TMEM buffer n & 1), B = K MN-major in smem
+      const uint64_t kd = ptx::desc_advance(k_desc_mn, (n % KS) * Geo::kTileBytes);
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc, tmem + kColDS + (n & 1) * 64 + kk * 8,
+                              ptx::desc_advance(kd, kk * 2048), idesc_o, (n > 0 || kk > 0) ? 1u : 0u);
+      ptx::mma_commit_warp(&k_empty[n % KS]);
     }
+    if (ok) ptx::mma_commit_warp(&acc_full);
+    ptx::mma_commit_warp(&mma_final);
+    ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    __syncwarp();
   } else {
     const int quad = warp & 3, half = warp >> 2;
     const int r = quad * 32 + lane;  // query row = TMEM lane

@@ -50,7 +50,7 @@ constexpr int kFwdThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther == kFwdThreads * kRegsLaunch,
               "register split must add up to the launch allocation");
-constexpr int kRing = 4;
+constexpr int kRingMax = 8;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -58,9 +58,13 @@ template <int D>
 struct FwdGeom {
   static constexpr int kQBytes = kBM * D * 2;   // one head's Q tile
   static constexpr int kKVBytes = kBN * D * 2;  // one K or V tile
+  // K/V ring depth: a K or V tile takes ~5000 cycles to arrive from L2 under full load, so
+  // each slot must be refilled about two tile periods ahead (5 x 32 KB for d = 128)
+  static constexpr int kRing = D == 128 ? 5 : kRingMax;
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kQBytes;
   static constexpr int kSmem = kOffRing + kRing * kKVBytes + 1024;  // + alignment slack
+  static_assert(kRing <= kRingMax && kSmem <= 227 * 1024, "shared memory budget");
   static constexpr int kColO = 256;
 };
 
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t kv_full[kRing], kv_empty[kRing];
+  __shared__ __align__(8) uint64_t kv_full[kRingMax], kv_empty[kRingMax];
   __shared__ __align__(8) uint64_t s_full[2], p_ready[2], o_done[2];
   __shared__ __align__(8) uint64_t mma_final;
   __shared__ uint32_t tmem_base_sh;
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&q_full, 1);
-    for (int s = 0; s < kRing; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
+    for (int s = 0; s < Geo::kRing; ++s) { ptx::mbar_init(&kv_full[s], 1); ptx::mbar_init(&kv_empty[s], 1); }
     for (int k = 0; k < 2; ++k) {
       ptx::mbar_init(&s_full[k], 1);
       ptx::mbar_init(&p_ready[k], 4);
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       cur.init(T);
       int issued = 0;
       for (int idx = 0; idx < 2 * ntiles; ++idx) {
-        const int s = idx % kRing;
-        if (idx >= kRing && !ptx::mbar_wait(&kv_empty[s], ((idx / kRing) - 1) & 1, &abort_flag, a.status)) break;
+        const int s = idx % Geo::kRing;
+        if (idx >= Geo::kRing && !ptx::mbar_wait(&kv_empty[s], ((idx / Geo::kRing) - 1) & 1, &abort_flag, a.status)) break;
         const bool is_v = idx & 1;
         uint8_t* dst = sRing + s * Geo::kKVBytes;
         ptx::mbar_arrive_expect_tx(&kv_full[s], Geo::kKVBytes);
@@ -156,82 +160,85 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       }
       // drain: no copy may still be landing in shared memory when the CTA exits
       ptx::mbar_wait(&q_full, 0, nullptr, a.status);
-      for (int idx = (issued > kRing ? issued - kRing : 0); idx < issued; ++idx)
-        ptx::mbar_wait(&kv_full[idx % kRing], (idx / kRing) & 1, nullptr, a.status);
+      for (int idx = (issued > Geo::kRing ? issued - Geo::kRing : 0); idx < issued; ++idx)
+        ptx::mbar_wait(&kv_full[idx % Geo::kRing], (idx / Geo::kRing) & 1, nullptr, a.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sQ), ring_addr = ptx::smem_u32(sRing);
-      const int nslot = has1 ? 2 : 1;
+    // The whole warp walks the issue loop (uniform operands); one elected lane issues each
+    // MMA and commit.  Descriptors are built once and advanced by constant offsets.
+    constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
+    constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
+    const uint64_t q_desc = ptx::smem_desc_sw128(ptx::smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = ptx::smem_desc_sw128(ptx::smem_u32(sRing), 16, 1024);
+    const uint64_t v_desc = ptx::smem_desc_sw128(ptx::smem_u32(sRing), 16384, 1024);
+    const int nslot = has1 ? 2 : 1;
 
-      auto issue_s = [&](int k, int kslot) {
-        const uint32_t qa = q_addr + k * Geo::kQBytes, kb = ring_addr + kslot * Geo::kKVBytes;
+    auto issue_s = [&](int k, int kslot) {
+      const uint64_t qd = ptx::desc_advance(q_desc, k * Geo::kQBytes);
+      const uint64_t kd = ptx::desc_advance(k_desc, kslot * Geo::kKVBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          ptx::mma_bf16_ss(tmem + k * 128, ptx::smem_desc_sw128(qa + off, 16, 1024),
-                           ptx::smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_k (+)= P_k V: P_k (bf16, in TMEM over the S_k columns) is the A operand
-      auto issue_pv = [&](int k, int vslot, bool accumulate) {
-        const uint32_t vb = ring_addr + vslot * Geo::kKVBytes;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        ptx::mma_bf16_ss_warp(tmem + k * 128, ptx::desc_advance(qd, off), ptx::desc_advance(kd, off), idesc_s,
+                              kk > 0 ? 1u : 0u);
+      }
+    };
+    // O_k (+)= P_k V: P_k (bf16, in TMEM over the S_k columns) is the A operand
+    auto issue_pv = [&](int k, int vslot, bool accumulate) {
+      const uint64_t vd = ptx::desc_advance(v_desc, vslot * Geo::kKVBytes);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + Geo::kColO + k * D, tmem + k * 128 + kk * 8,
-                           ptx::smem_desc_sw128(vb + kk * 2048, 16384, 1024), idesc_o,
-                           (accumulate || kk > 0) ? 1u : 0u);
-      };
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColO + k * D, tmem + k * 128 + kk * 8, ptx::desc_advance(vd, kk * 2048),
+                              idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+    };
 
-      bool ok = ptx::mbar_wait(&q_full, 0, &abort_flag, a.status);
+    bool ok = ptx::mbar_wait_warp(&q_full, 0, &abort_flag, a.status);
+    ptx::tc_fence_after();
+    for (int n = 0; ok && n < ntiles; ++n) {
+      const int kidx = 2 * n, vidx = 2 * n + 1;
+      const int kslot = kidx % Geo::kRing, vslot = vidx % Geo::kRing;
+      if (!(ok = ptx::mbar_wait_warp(&kv_full[kslot], (kidx / Geo::kRing) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
-      for (int n = 0; ok && n < ntiles; ++n) {
-        const int kidx = 2 * n, vidx = 2 * n + 1;
-        const int kslot = kidx % kRing, vslot = vidx % kRing;
-        if (!(ok = ptx::mbar_wait(&kv_full[kslot], (kidx / kRing) & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        // S0(n): P0(n-1) was consumed by PV0(n-1), issued earlier
-        issue_s(0, kslot);
-        ptx::mma_commit(&s_full[0]);
-        if (nslot == 2) {
-          // PV1(n-1): overlaps with softmax 0 working on S0(n)
-          if (n > 0) {
-            const int pv = 2 * (n - 1) + 1;
-            if (!(ok = ptx::mbar_wait(&p_ready[1], (n - 1) & 1, &abort_flag, a.status))) break;
-            ptx::tc_fence_after();
-            issue_pv(1, pv % kRing, n - 1 > 0);
-            ptx::mma_commit(&kv_empty[pv % kRing]);
-          }
-          issue_s(1, kslot);
-          ptx::mma_commit(&s_full[1]);
+      // S0(n): P0(n-1) was consumed by PV0(n-1), issued earlier
+      issue_s(0, kslot);
+      ptx::mma_commit_warp(&s_full[0]);
+      if (nslot == 2) {
+        // PV1(n-1): overlaps with softmax 0 working on S0(n)
+        if (n > 0) {
+          const int pv = 2 * (n - 1) + 1;
+          if (!(ok = ptx::mbar_wait_warp(&p_ready[1], (n - 1) & 1, &abort_flag, a.status))) break;
+          ptx::tc_fence_after();
+          issue_pv(1, pv % Geo::kRing, n - 1 > 0);
+          ptx::mma_commit_warp(&kv_empty[pv % Geo::kRing]);
         }
-        ptx::mma_commit(&kv_empty[kslot]);
-        // PV0(n)
-        if (!(ok = ptx::mbar_wait(&kv_full[vslot], (vidx / kRing) & 1, &abort_flag, a.status))) break;
-        if (!(ok = ptx::mbar_wait(&p_ready[0], n & 1, &abort_flag, a.status))) break;
-        ptx::tc_fence_after();
-        issue_pv(0, vslot, n > 0);
-        if (nslot == 1) ptx::mma_commit(&kv_empty[vslot]);
+        issue_s(1, kslot);
+        ptx::mma_commit_warp(&s_full[1]);
       }
-      if (ok && ntiles > 0) {
-        ptx::mma_commit(&o_done[0]);
-        if (nslot == 2) {
-          const int n = ntiles - 1, pv = 2 * n + 1;
-          if (ptx::mbar_wait(&p_ready[1], n & 1, &abort_flag, a.status)) {
-            ptx::tc_fence_after();
-            issue_pv(1, pv % kRing, n > 0);
-            ptx::mma_commit(&kv_empty[pv % kRing]);
-            ptx::mma_commit(&o_done[1]);
-          }
-        }
-      }
-      // all issued MMAs complete before TMEM can be released
-      ptx::mma_commit(&mma_final);
-      ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+      ptx::mma_commit_warp(&kv_empty[kslot]);
+      // PV0(n)
+      if (!(ok = ptx::mbar_wait_warp(&kv_full[vslot], (vidx / Geo::kRing) & 1, &abort_flag, a.status))) break;
+      if (!(ok = ptx::mbar_wait_warp(&p_ready[0], n & 1, &abort_flag, a.status))) break;
+      ptx::tc_fence_after();
+      issue_pv(0, vslot, n > 0);
+      if (nslot == 1) ptx::mma_commit_warp(&kv_empty[vslot]);
     }
+    if (ok && ntiles > 0) {
+      ptx::mma_commit_warp(&o_done[0]);
+      if (nslot == 2) {
+        const int n = ntiles - 1, pv = 2 * n + 1;
+        if (ptx::mbar_wait_warp(&p_ready[1], n & 1, &abort_flag, a.status)) {
+          ptx::tc_fence_after();
+          issue_pv(1, pv % Geo::kRing, n > 0);
+          ptx::mma_commit_warp(&kv_empty[pv % Geo::kRing]);
+          ptx::mma_commit_warp(&o_done[1]);
+        }
+      }
+    }
+    // all issued MMAs complete before TMEM can be released
+    ptx::mma_commit_warp(&mma_final);
+    ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
+    __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
