@@ -459,38 +459,100 @@ def run_cowa(args, world, rank, local):
                     "algorithmic": f"{work:.4e} visible K/V bytes per call"}
     roofline["all_kernels_ms"] = {kname: v[0] for kname, v in kernels.items()}
 
-    # ---- end to end: host buffers, copies inside the timed region
+    # ---- end to end: host buffers, copies inside the timed region.  Every step copies its inputs
+    # (q, k, v, dO of the layer, q_t and pos of the decode; the KV cache is resident device state)
+    # in from pinned host memory and its results (o, dq, dk, dv, decode o) out to pinned host
+    # memory.  Steps are pipelined the way a training or serving loop prefetches: three streams
+    # (copy-in, compute, copy-out) and two device buffer sets, so step i+1's inputs land while
+    # step i computes and step i's results leave while step i+1 computes.  Within a step the
+    # forward starts once q, k, v are in (dO lands meanwhile), o leaves while the backward runs.
     e2e = None
     if not args.no_e2e:
         pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-        h_in = [pin(x) for x in (q, k, v, do, qt)]
-        for hsrc, dsrc in zip(h_in, (q, k, v, do, qt)):
-            hsrc.copy_(dsrc)
+        names_in = ("q", "k", "v", "do", "qt")
+        h_in = {n: pin(x) for n, x in zip(names_in, (q, k, v, do, qt))}
+        for n, x in zip(names_in, (q, k, v, do, qt)):
+            h_in[n].copy_(x)
         h_pos = pos.cpu().pin_memory()
-        h_out = [pin(x) for x in (o, dq, dk, dv, od)]
-        h2d = sum(x.numel() * x.element_size() for x in h_in) + h_pos.numel() * 4
-        d2h = sum(x.numel() * x.element_size() for x in h_out)
-        KE = max(1, min(K, 3))
+        names_out = ("o", "dq", "dk", "dv", "od")
+        h_out = {n: pin(x) for n, x in zip(names_out, (o, dq, dk, dv, od))}
+        h2d = sum(x.numel() * x.element_size() for x in h_in.values()) + h_pos.numel() * 4
+        d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
-        def e2e_step():
-            for hsrc, ddst in zip(h_in, (q, k, v, do, qt)):
-                ddst.copy_(hsrc, non_blocking=True)
-            pos.copy_(h_pos, non_blocking=True)
-            fwd(); bwd(); dec()
-            for ddst, hsrc in zip(h_out, (o, dq, dk, dv, od)):
-                ddst.copy_(hsrc, non_blocking=True)
+        def buffer_set():
+            st = {n: torch.empty_like(x) for n, x in zip(names_in + ("pos",), (q, k, v, do, qt, pos))}
+            st.update({n: torch.empty_like(x) for n, x in zip(names_out + ("lse", "lsed"), (o, dq, dk, dv, od, lse, lsed))})
+            st.update({n: torch.zeros_like(x) for n, x in (("ws_f", ws_f), ("ws_b", ws_b), ("ws_d", ws_d))})
+            return st
 
-        e2e_step(); torch.cuda.synchronize()
+        sets = [buffer_set(), buffer_set()]
+        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        inputs_free = [None, None]   # compute of the step that last used the set has read its inputs
+        outputs_free = [None, None]  # copy-out of the step that last used the set is done
+        new_ev = lambda: torch.cuda.Event()
+
+        def e2e_step(i):
+            st = sets[i % 2]
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if inputs_free[j] is not None:
+                    s_in.wait_event(inputs_free[j])
+                for n in ("q", "k", "v"):
+                    st[n].copy_(h_in[n], non_blocking=True)
+                e_qkv = new_ev(); e_qkv.record(s_in)
+                st["do"].copy_(h_in["do"], non_blocking=True)
+                e_do = new_ev(); e_do.record(s_in)
+                st["qt"].copy_(h_in["qt"], non_blocking=True)
+                st["pos"].copy_(h_pos, non_blocking=True)
+                e_dec_in = new_ev(); e_dec_in.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(e_qkv)
+                if outputs_free[j] is not None:
+                    s_cmp.wait_event(outputs_free[j])
+                cw.cowa_fwd(st["q"], st["k"], st["v"], pat, out=st["o"], lse=st["lse"], workspace=st["ws_f"])
+                e_fwd = new_ev(); e_fwd.record(s_cmp)
+                s_cmp.wait_event(e_do)
+                cw.cowa_bwd(st["q"], st["k"], st["v"], st["o"], st["lse"], st["do"], pat, dq=st["dq"], dk=st["dk"],
+                            dv=st["dv"], workspace=st["ws_b"])
+                e_bwd = new_ev(); e_bwd.record(s_cmp)
+                s_cmp.wait_event(e_dec_in)
+                cw.cowa_decode(st["qt"], kc, vc, st["pos"], dpat, out=st["od"], lse=st["lsed"], workspace=st["ws_d"])
+                e_cmp = new_ev(); e_cmp.record(s_cmp)
+                inputs_free[j] = e_cmp
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(e_fwd)
+                h_out["o"].copy_(st["o"], non_blocking=True)
+                s_out.wait_event(e_bwd)
+                for n in ("dq", "dk", "dv"):
+                    h_out[n].copy_(st[n], non_blocking=True)
+                s_out.wait_event(e_cmp)
+                h_out["od"].copy_(st["od"], non_blocking=True)
+                e_o = new_ev(); e_o.record(s_out)
+                outputs_free[j] = e_o
+
+        KE = max(2, min(K, 10))
+        e2e_step(0); e2e_step(1); torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(KE):
-            e2e_step()
-        b.record(); torch.cuda.synchronize()
+        main_s = torch.cuda.current_stream(dev)
+        a.record(main_s)
+        for st_ in (s_in, s_cmp, s_out):
+            st_.wait_stream(main_s)
+        for i in range(KE):
+            e2e_step(i)
+        for st_ in (s_in, s_cmp, s_out):
+            main_s.wait_stream(st_)
+        b.record(main_s); torch.cuda.synchronize()
         barrier()
+        for st_ in sets:
+            for n in ("ws_f", "ws_b", "ws_d"):
+                if cw.workspace_status(st_[n]) != 0:
+                    raise RuntimeError("device status set during the end-to-end steps")
         e_ms = maxr(a.elapsed_time(b)) / KE
         e2e = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
+               "pipelined": "copy-in / compute / copy-out streams, two device buffer sets"}
+        del sets
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:

@@ -22,9 +22,11 @@
 // grows by more than 2^8; the final division uses the same stale max, so the result is
 // exact).  P is rounded to bf16 and written back into TMEM over the S columns it came from,
 // where the P V MMA reads it as its A operand (no shared-memory round trip).  fp32
-// accumulation throughout.  Exponentials run on the special-function unit; COWA_FWD_POLY_MASK
-// can move a share of them to an FMA-pipe polynomial (exp2_poly.cuh), which measured slower
-// on B200 for this kernel (its softmax is bound by instruction issue), so it is off.
+// accumulation throughout.  Exponentials run on the special-function unit (an FMA-pipe
+// polynomial share measured slower on B200 here).  Each tile's exponentials use the running
+// max from before the tile while the tile's own max is gathered in the same pass; the tile is
+// redone only when that max grows the running one past the rescale threshold, so the common
+// path never waits for a row reduction and gives the same bits as max-first.
 //
 // MMA order per KV tile n: S0(n), PV1(n-1), S1(n), PV0(n).  Softmax 0 works on S0(n) while
 // the tensor core runs PV1(n-1) and S1(n), softmax 1 on S1(n) during PV0(n) and S0(n+1).
@@ -35,10 +37,7 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
-#include <type_traits>
-
 #include "cowa_internal.h"
-#include "exp2_poly.cuh"
 #include "kernel_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -67,13 +66,6 @@ struct FwdGeom {
   static_assert(kRing <= kRingMax && kSmem <= 227 * 1024, "shared memory budget");
   static constexpr int kColO = 256;
 };
-
-// Exponentials of columns c with bit (c & 7) of the mask set go to the FMA pipe (exp2_poly.cuh);
-// e.g. 0x52 = columns 1, 4, 6 of every 8.  Off by default (see above).
-#ifndef COWA_FWD_POLY_MASK
-#define COWA_FWD_POLY_MASK 0x00
-#endif
-__device__ __forceinline__ constexpr bool poly_col(int c) { return ((COWA_FWD_POLY_MASK >> (c & 7)) & 1) != 0; }
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_constant__ FwdArgs a) {
@@ -261,62 +253,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         const bool need_mask = (s0 + kBN > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kBN));
         if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
-        uint32_t xr[128];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) ptx::tmem_ld32(s_tm + q * 32, xr + q * 32);
-        ptx::tmem_wait_ld();
         // visible key columns of row t within [s0, s0+128), relative to s0 (partial tiles only)
         const int sink_end = imin(a.pat.S, t + 1) - s0;
         const int band_lo = imax(0, t - a.pat.L + 1) - s0;
         const int diag_end = t + 1 - s0;
         const int lr_lo = iv.lo - s0, lr_hi = imin(iv.hi, t + 1) - s0;
+        uint32_t xr[128];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ptx::tmem_ld32(s_tm + q * 32, xr + q * 32);
+        ptx::tmem_wait_ld();
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
             const bool vis = (c < sink_end) || (c >= band_lo && c < diag_end) || (c >= lr_lo && c < lr_hi);
-            if (!vis) xr[c] = 0xff800000u;  // -inf
+            if (!vis) xr[c] = 0xff800000u;  // -inf: gives exactly 0
           }
         }
-        // row max as a shallow tree (8 independent partial maxima), not a 64-deep chain
-        float pm[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pm[e] = fmaxf(__uint_as_float(xr[e]), __uint_as_float(xr[e + 8]));
-#pragma unroll
-        for (int c = 16; c < 128; c += 16)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) pm[e] = ptx::fmax3(pm[e], __uint_as_float(xr[c + e]), __uint_as_float(xr[c + 8 + e]));
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-        const float m_new = fmaxf(m_used, mx * sl2);
-        // lazy rescale: only when the running max grows by more than 2^8 (or first finite max);
-        // PV_k(n-1) has completed (the commit of S_k(n) covers it), so O_k is stable here
-        const bool grow = (m_new != -INFINITY) && (m_used == -INFINITY || m_new > m_used + kRescaleThreshold);
-        float alpha = 1.f;
-        if (grow) {
-          alpha = ptx::ex2(m_used - m_new);  // 0 when nothing was visible before
-          m_used = m_new;
-          lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
-        }
-        if (n > 0 && __any_sync(0xffffffffu, grow)) {
-          // O row *= alpha, a warp-collective TMEM round trip (alpha = 1 on the other lanes)
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(o_tm + c * 32, ov);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            ptx::tmem_st32(o_tm + c * 32, ov);
-          }
-        }
-        const float m_eff = m_used == -INFINITY ? 0.f : m_used;
-        const uint64_t negm = ptx::f2_pack(-m_eff, -m_eff);
+        // P = 2^(s*scale*log2e - m) with m the running max from before this tile, rounded to
+        // bf16 and written back into TMEM over the S columns (the A operand of P V); the tile's
+        // row max is gathered in the same pass.  Only when that max grows the running one by
+        // more than 2^8 (lazy rescale; rare after the first tiles) is the tile redone with the
+        // new max, so the common path never waits for the row reduction.
         uint64_t ts[4];  // this tile's row sum, 4 independent packed accumulators
+        float pm[8];     // partial row maxima
+        auto pass = [&](float m) {
+          const uint64_t negm = ptx::f2_pack(-m, -m);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) ts[e] = ptx::f2_pack(0.f, 0.f);
-        // P = 2^(s*scale*log2e - m), rounded to bf16, back into TMEM over the S columns
-        // (masked scores are -inf and give exactly 0).  Two instantiations so that the
-        // FMA-pipe share (unmasked tiles only) is decided at compile time per loop.
-        auto exp_tile = [&](auto fma_share) {
+          for (int e = 0; e < 4; ++e) ts[e] = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint32_t pw[32];
@@ -326,23 +289,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
               float e0, e1;
               ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(xr[c]), __uint_as_float(xr[c + 1])), sl2x2, negm),
                              e0, e1);
-              float p0, p1;
-              if (decltype(fma_share)::value && poly_col(c) && poly_col(c + 1)) {
-                exp2_fma_x2(e0, e1, p0, p1);  // a pair on the FMA pipe
-              } else {
-                p0 = (decltype(fma_share)::value && poly_col(c)) ? exp2_fma(e0) : ptx::ex2(e0);
-                p1 = (decltype(fma_share)::value && poly_col(c + 1)) ? exp2_fma(e1) : ptx::ex2(e1);
-              }
+              const float p0 = ptx::ex2(e0), p1 = ptx::ex2(e1);
               ts[c2 & 3] = ptx::f2_add(ts[c2 & 3], ptx::f2_pack(p0, p1));
               pw[c2] = ptx::pack_bf16(p0, p1);
             }
             ptx::tmem_st32(s_tm + 32 * h, pw);
           }
         };
-        if (COWA_FWD_POLY_MASK == 0 || need_mask)
-          exp_tile(std::false_type{});
-        else
-          exp_tile(std::true_type{});
+        pass(m_used == -INFINITY ? 0.f : m_used);
+        // row max (independent of the exponentials above, so it overlaps them)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pm[e] = fmaxf(__uint_as_float(xr[e]), __uint_as_float(xr[e + 8]));
+#pragma unroll
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pm[e] = ptx::fmax3(pm[e], __uint_as_float(xr[c + e]), __uint_as_float(xr[c + 8 + e]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        const float m_new = fmaxf(m_used, mx * sl2);
+        const bool grow = (m_new != -INFINITY) && (m_used == -INFINITY || m_new > m_used + kRescaleThreshold);
+        if (__any_sync(0xffffffffu, grow)) {
+          float alpha = 1.f;
+          if (grow) {
+            alpha = ptx::ex2(m_used - m_new);  // 0 when nothing was visible before
+            m_used = m_new;
+            lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
+          }
+          if (n > 0) {
+            // O row *= alpha, a warp-collective TMEM round trip (alpha = 1 on the other lanes);
+            // PV_k(n-1) has completed (the commit of S_k(n) covers it), so O_k is stable here
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t ov[32];
+              ptx::tmem_ld32(o_tm + c * 32, ov);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              ptx::tmem_st32(o_tm + c * 32, ov);
+            }
+          }
+          // redo the tile from the scores still in registers (lanes whose max did not grow
+          // recompute the same values); the stores replace the speculative P
+          ptx::tmem_wait_st();
+          pass(m_used == -INFINITY ? 0.f : m_used);
+        }
         lsum = ptx::f2_add(lsum, ptx::f2_add(ptx::f2_add(ts[0], ts[1]), ptx::f2_add(ts[2], ts[3])));
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
