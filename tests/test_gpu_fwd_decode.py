@@ -70,6 +70,26 @@ def test_fwd_strided_inputs(cuda_device):
     assert np.abs(lse.cpu().numpy() - want_l).max() <= LSE_ATOL
 
 
+def test_fwd_running_max_growth(cuda_device):
+    """Scores that jump in a later tile: keys of some tiles scaled up so that the running row
+    max grows by far more than the lazy-rescale threshold after the first tile (rescale of O
+    and a redone tile), next to the reverse case (large sink keys: no growth after tile 0)."""
+    B, N, Hq, Hkv, d = 1, 1000, 4, 2, 128
+    pat = cw.Pattern(16, 512, 1000, 2)
+    q64, q = host_and_device((B, N, Hq, d), "q", cuda_device, 11)
+    _, k = host_and_device((B, N, Hkv, d), "k", cuda_device, 11)
+    v64, v = host_and_device((B, N, Hkv, d), "v", cuda_device, 11)
+    for lo, hi, f in [(768, 1000, 6.0), (0, 16, 6.0), (300, 420, 4.0)]:
+        k2 = k.clone()
+        k2[:, lo:hi] = (k2[:, lo:hi].float() * f).to(torch.bfloat16)
+        o, lse = cw.cowa_fwd(q, k2, v, pat)
+        torch.cuda.synchronize()
+        want_o, want_l = orc.attention_fwd(q64, to64(k2), v64, oracle_pattern(pat))
+        err_o = np.abs(to64(o) - want_o).max()
+        err_l = np.abs(lse.cpu().numpy().astype(np.float64) - want_l).max()
+        assert err_o <= O_ATOL and err_l <= LSE_ATOL, (lo, hi, err_o, err_l)
+
+
 def _check_fwd_rows(B, N, Hq, Hkv, d, pat, device, rows, batches, use_cuda_gen=False):
     if use_cuda_gen:
         q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), device)
