@@ -352,8 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   // ds_ready is per dS buffer: a barrier can then never run two phases ahead of its waiter
-  __shared__ __align__(8) uint64_t q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, consumed,
-      ds_ready[2], acc_full, mma_final;
+  // consumed_s / consumed_dp: the softmax holds S / dP of the tile in registers, so the next
+  // tile's S / dP MMAs may overwrite their columns (S can start before dP has been read)
+  __shared__ __align__(8) uint64_t q_full, k_full[3], k_empty[3], v_full[2], v_empty[2], sdp_full, consumed_s,
+      consumed_dp, ds_ready[2], acc_full, mma_final;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -381,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     for (int s = 0; s < KS; ++s) { ptx::mbar_init(&k_full[s], 1); ptx::mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < VS; ++s) { ptx::mbar_init(&v_full[s], 1); ptx::mbar_init(&v_empty[s], 1); }
     ptx::mbar_init(&sdp_full, 1);
-    ptx::mbar_init(&consumed, kComputeWarps);
+    ptx::mbar_init(&consumed_s, kComputeWarps);
+    ptx::mbar_init(&consumed_dp, kComputeWarps);
     ptx::mbar_init(&ds_ready[0], kComputeWarps);
     ptx::mbar_init(&ds_ready[1], kComputeWarps);
     ptx::mbar_init(&acc_full, 1);
@@ -440,18 +443,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     const uint64_t k_desc = ptx::smem_desc_sw128(ptx::smem_u32(sK), 16, 1024);
     const uint64_t k_desc_mn = ptx::smem_desc_sw128(ptx::smem_u32(sK), 16384, 1024);
     const uint64_t v_desc = ptx::smem_desc_sw128(ptx::smem_u32(sV), 16, 1024);
-    // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns; V_n is free afterwards
+    // S = Q K^T and dP = dO V^T of KV tile n into the S / dP columns; V_n is free afterwards.
+    // For n > 0 each half waits until the softmax has read that half of tile n-1.
     auto issue_sdp = [&](int n) -> bool {
+      if (n > 0 && !ptx::mbar_wait_warp(&consumed_s, (n - 1) & 1, &abort_flag, a.status)) return false;
       if (!ptx::mbar_wait_warp(&k_full[n % KS], (n / KS) & 1, &abort_flag, a.status)) return false;
-      if (!ptx::mbar_wait_warp(&v_full[n % VS], (n / VS) & 1, &abort_flag, a.status)) return false;
       ptx::tc_fence_after();
       const uint64_t kd = ptx::desc_advance(k_desc, (n % KS) * Geo::kTileBytes);
-      const uint64_t vd = ptx::desc_advance(v_desc, (n % VS) * Geo::kTileBytes);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
         ptx::mma_bf16_ss_warp(tmem + 0, ptx::desc_advance(q_desc, off), ptx::desc_advance(kd, off), idesc_s, kk > 0);
       }
+      if (n > 0 && !ptx::mbar_wait_warp(&consumed_dp, (n - 1) & 1, &abort_flag, a.status)) return false;
+      if (!ptx::mbar_wait_warp(&v_full[n % VS], (n / VS) & 1, &abort_flag, a.status)) return false;
+      ptx::tc_fence_after();
+      const uint64_t vd = ptx::desc_advance(v_desc, (n % VS) * Geo::kTileBytes);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -466,8 +473,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     if (ok && ntiles > 0) ok = issue_sdp(0);
     for (int n = 0; ok && n < ntiles; ++n) {
       // the softmax holds S(n), dP(n) in registers: compute the next tile's S and dP now
-      if (!(ok = ptx::mbar_wait_warp(&consumed, n & 1, &abort_flag, a.status))) break;
-      ptx::tc_fence_after();
       if (n + 1 < ntiles && !(ok = issue_sdp(n + 1))) break;
       if (!(ok = ptx::mbar_wait_warp(&ds_ready[n & 1], (n >> 1) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
@@ -506,12 +511,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       uint32_t sv[64], pv[64];
       ptx::tmem_ld32(lane_base + half * 64, sv);
       ptx::tmem_ld32(lane_base + half * 64 + 32, sv + 32);
-      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);
+      ptx::tmem_wait_ld();
+      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);  // in flight while S is released
       ptx::tmem_ld32(lane_base + 128 + half * 64 + 32, pv + 32);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&consumed_s);  // S columns may be overwritten now
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&consumed);  // S / dP columns may be overwritten now
+      if (lane == 0) ptx::mbar_arrive(&consumed_dp);  // dP columns too
       const bool use_poly = !need_mask && t < a.N;
       // dS buffer n & 1 was last read by dQ(n-2), which the commit of S(n) covers.  The element
       // loop is instantiated with and without the mask, chosen once per tile.
