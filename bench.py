@@ -7,7 +7,8 @@ Prints one JSON line (rank 0).  `value` is visible TFLOP/s of the training part
 (forward 4*d and backward 10*d FLOPs per visible query-key pair, summed over all
 ranks) divided by the max-over-ranks device time of the whole step (decode
 included); `parts` gives each call's CUDA-event time, the decode GB/s over the
-visible K/V bytes, and the same for the dense-causal mode when --dense is given.
+visible K/V bytes, and the same for the dense-causal mode when --dense is given;
+--sweep adds the other configurations (see `sweep_configs`).
 Inputs are larger than L2 (126 MB), so no flush is needed between steps.
 
 N > 1: one process per GPU (torchrun); every rank runs the same per-GPU workload on
@@ -259,6 +260,85 @@ def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
     return done_flops / t_used / 1e12, desc, threads, t_used
 
 
+# ------------------------------------------------------------------------------ sweep
+SWEEP = [  # (name, B, N, Hq, Hkv, d, S, L, T, D, bwd)
+    ("prefill 8K D=8", 2, 8192, 32, 8, 128, 128, 1024, 8192, 8, True),
+    ("prefill 8K D=4", 2, 8192, 32, 8, 128, 128, 1024, 8192, 4, False),
+    ("prefill 8K D=2", 2, 8192, 32, 8, 128, 128, 1024, 8192, 2, False),
+    ("prefill 8K D=1", 2, 8192, 32, 8, 128, 128, 1024, 8192, 1, False),
+    ("train 32K dense causal", 1, 32768, 40, 8, 128, 128, 32768, 32768, 8, True),
+    ("long 128K", 1, 131072, 40, 8, 128, 128, 4096, 131072, 8, True),
+    ("long 128K dense causal", 1, 131072, 40, 8, 128, 128, 131072, 131072, 8, True),
+]
+
+
+def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
+    """Times cowa_fwd and the three backward stages on each SWEEP configuration and the decode
+    step in the dense-causal mode, CUDA events, median of `reps` after one warm-up.  Fractions
+    are of the measured burst bf16 peak (each kernel runs alone) and of the HBM copy rate."""
+    import torch
+
+    from structured_sparse_attention_cowa_b200 import cowa as cw
+    from structured_sparse_attention_cowa_b200 import synth
+
+    out = []
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); fn(); b.record(); torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    for name, B, N, Hq, Hkv, d, S, L, T, D, do_bwd in SWEEP:
+        pat = cw.Pattern(S, L, T, D)
+        q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), dev)
+        k = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("k"), dev)
+        v = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("v"), dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        pairs = visible_pairs(N, S, L, T, D, Hkv, Hq, B)
+        f_ms = timed(lambda: cw.cowa_fwd(q, k, v, pat, out=o, lse=lse))
+        row = {"config": name, "B": B, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "S": S, "L": L, "T": T, "D": D,
+               "visible_pairs": pairs, "fwd_ms": f_ms, "fwd_tflops": 4.0 * d * pairs / (f_ms * 1e-3) / 1e12}
+        row["fwd_frac_burst"] = row["fwd_tflops"] / peak_tf
+        if do_bwd:
+            do = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("do"), dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            import ctypes
+
+            n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+            ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+            stage = lambda st: cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws, stages=st)
+            st_ms = {nm: timed(lambda st=st: stage(st)) for nm, st in
+                     (("preprocess", cw.BWD_PREPROCESS), ("dkdv", cw.BWD_DKDV), ("dq", cw.BWD_DQ))}
+            b_ms = sum(st_ms.values())
+            row.update({"bwd_ms": b_ms, "bwd_stages_ms": st_ms, "bwd_tflops": 10.0 * d * pairs / (b_ms * 1e-3) / 1e12})
+            row["bwd_frac_burst"] = row["bwd_tflops"] / peak_tf
+            if cw.workspace_status(ws) != 0:
+                raise RuntimeError(f"device status set in sweep config {name}")
+            del do, dq, dk, dv, ws
+        out.append(row)
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+
+    # decode in the dense-causal mode: every cached token up to pos is visible
+    dc = DECODE
+    dpat = cw.Pattern(dc["S"], dc["T"], dc["T"], dc["D"])
+    qt = synth.cuda_normal_bf16((dc["B"], dc["Hq"], dc["d"]), synth.seed_of("q_t"), dev)
+    pos = torch.full((dc["B"],), dc["pos"], dtype=torch.int32, device=dev)
+    od = torch.empty((dc["B"], dc["Hq"], dc["d"]), dtype=torch.bfloat16, device=dev)
+    d_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, dpat, out=od))
+    dbytes = float(dc["pos"] + 1) * dc["B"] * dc["Hkv"] * dc["d"] * 2 * 2
+    out.append({"config": "decode 128K dense causal", "B": dc["B"], "pos": dc["pos"], "decode_ms": d_ms,
+                "decode_gbs": dbytes / (d_ms * 1e-3) / 1e9, "decode_frac_hbm": dbytes / (d_ms * 1e-3) / 1e9 / hbm_gbs,
+                "bytes": dbytes})
+    return out
+
+
 # ------------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -269,6 +349,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dense", action="store_true", help="also time the dense-causal mode (L >= T)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time the other configurations (8K prefill D sweep, 128K layer, dense-causal at "
+                         "32K/128K, dense decode) and add them under 'sweep' (one GPU only)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -560,6 +643,10 @@ def run_cowa(args, world, rank, local):
         cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
                "host_cpus": os.cpu_count()}
 
+    sweep = None
+    if args.sweep and world == 1:
+        sweep = sweep_configs(dev, kc, vc, burst, hbm)  # each kernel timed alone: burst peak
+
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
@@ -572,6 +659,8 @@ def run_cowa(args, world, rank, local):
                        "parallelism": f"batch-sharded x{world} (weak)"},
             "parts": parts, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": K * 6, "clocks": clk.summary()}  # fwd 1 + bwd 3 + decode 2 per step
+    if sweep is not None:
+        line["sweep"] = sweep
     print(json.dumps(line), flush=True)
     return 0
 
