@@ -97,6 +97,21 @@ cowa_status cowa_fwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, i
                      cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, float* lse,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---- chunked prefill: a block of queries against keys already written -------------------
+ * The same operation for the query rows at positions q_offset .. q_offset+N_q-1 against the
+ * keys at positions 0 .. N_k-1.  The pattern is position arithmetic applied the same way in
+ * training and inference (skillfed.io news summary of CoWindow Attention, paragraph 2), so a later
+ * block of queries over a cache sees exactly the keys it would see in one full pass.  cowa_fwd is this call with q_offset = 0, N_q = N_k = N.
+ * Inputs  q [B, N_q, H_q, d]; k and v hold keys 0 .. N_k-1 (any cowa_tensor strides: a cache in
+ *         [B, H_kv, T_cap, d] layout is stride_t = d, stride_h = T_cap*d, stride_b = H_kv*T_cap*d)
+ * Outputs o [B, N_q, H_q, d] bf16; lse fp32 contiguous [B, H_q, N_q].
+ * Requires q_offset >= 0 and q_offset + N_q <= N_k (the block's own keys are present), else
+ * COWA_ERR_INVALID_ARG before any launch.  Workspace: cowa_fwd_workspace_size with N = N_q.
+ * Ownership, ordering and errors as for cowa_fwd. */
+cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int q_offset, int H_q, int H_kv,
+                           int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
 /* ---- backward ---------------------------------------------------------------------------
  * Gradients of sum(dO * O) for the forward above, from the saved o and lse.
  * Inputs  q, k, v, o, lse as produced/consumed by cowa_fwd; dO [B, N, H_q, d] bf16.

@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.cowa_fwd_workspace_size.restype = sz
     L.cowa_fwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, vp, sz, vp]
     L.cowa_fwd.restype = i
+    L.cowa_fwd_chunk.argtypes = [P, i, i, i, i, i, i, i, T, T, T, T, vp, vp, sz, vp]
+    L.cowa_fwd_chunk.restype = i
     L.cowa_bwd_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_bwd_workspace_size.restype = sz
     L.cowa_bwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
@@ -161,6 +163,43 @@ def cowa_fwd(q, k, v, pattern: Pattern, out=None, lse=None, workspace=None, stre
         workspace = _workspace(ws_bytes, q.device)
     _check("cowa_fwd", L.cowa_fwd(ctypes.byref(pat), B, N, Hq, Hkv, d, _t4(q), _t4(k), _t4(v), _t4(out),
                                   lse.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def cowa_fwd_chunk(q, k, v, pattern: Pattern, q_offset: int, n_k=None, kv_layout: str = "bthd", out=None,
+                   lse=None, workspace=None, stream=None):
+    """Chunked prefill: o [B,N_q,H_q,d] bf16 and lse [B,H_q,N_q] fp32 for the query rows at
+    positions q_offset .. q_offset+N_q-1 against the keys 0 .. n_k-1 of k, v.  k, v are
+    [B, N_k, H_kv, d] (kv_layout "bthd") or a cache [B, H_kv, T_cap, d] ("bhtd"); n_k defaults
+    to their full length and must cover q_offset + N_q."""
+    import torch
+
+    for n_, x_ in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n_, x_)
+    B, Nq, Hq, d = q.shape
+    if kv_layout == "bthd":
+        kt, vt = k, v
+    elif kv_layout == "bhtd":
+        kt, vt = k.transpose(1, 2), v.transpose(1, 2)  # strided views [B, T, H, d]
+    else:
+        raise ValueError("kv_layout is 'bthd' or 'bhtd'")
+    Hkv = kt.shape[2]
+    if n_k is None:
+        n_k = kt.shape[1]
+    if not 0 < n_k <= kt.shape[1]:
+        raise ValueError("n_k out of range")
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_fwd_workspace_size(ctypes.byref(pat), B, Nq, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q.device)
+    _check("cowa_fwd_chunk", L.cowa_fwd_chunk(ctypes.byref(pat), B, Nq, int(n_k), int(q_offset), Hq, Hkv, d, _t4(q),
+                                              _t4(kt), _t4(vt), _t4(out), lse.data_ptr(), workspace.data_ptr(),
+                                              workspace.numel(), _stream(stream)))
     return out, lse
 
 

@@ -184,27 +184,35 @@ size_t cowa_fwd_workspace_size(const cowa_pattern* pat, int B, int N, int Hq, in
 
 cowa_status cowa_fwd(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d, cowa_tensor q, cowa_tensor k,
                      cowa_tensor v, cowa_tensor o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return cowa_fwd_chunk(pat, B, N, N, 0, Hq, Hkv, d, q, k, v, o, lse, ws, ws_bytes, stream);
+}
+
+cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int q_offset, int Hq, int Hkv, int d,
+                           cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, float* lse, void* ws,
+                           size_t ws_bytes, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
-  COWA_TRY(check_heads(B, N, Hq, Hkv, d));
+  COWA_TRY(check_heads(B, N_q, Hq, Hkv, d));
+  if (q_offset < 0 || N_k < 1 || (int64_t)q_offset + N_q > (int64_t)N_k) return COWA_ERR_INVALID_ARG;
   COWA_TRY(check_tensor(q));
   COWA_TRY(check_tensor(k));
   COWA_TRY(check_tensor(v));
   COWA_TRY(check_tensor(o));
   if (!lse) return COWA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return COWA_ERR_ALIGNMENT;
-  COWA_TRY(check_ws(ws, ws_bytes, cowa_fwd_workspace_size(pat, B, N, Hq, Hkv, d)));
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_fwd_workspace_size(pat, B, N_q, Hq, Hkv, d)));
 
   FwdArgs a;
   memset(&a, 0, sizeof(a));
-  a.pat = p; a.B = B; a.N = N; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.pat = p; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.Nq = N_q; a.Nk = N_k; a.q_off = q_offset;
   a.o = o.ptr; a.o_sb = o.stride_b; a.o_st = o.stride_t; a.o_sh = o.stride_h;
   a.lse = lse;
   a.status = reinterpret_cast<uint32_t*>(ws);
   a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f;
-  if (!make_tmap_bf16(&a.tm_q, q.ptr, d, N, Hq, B, q.stride_t, q.stride_h, q.stride_b, 128) ||
-      !make_tmap_bf16(&a.tm_k, k.ptr, d, N, Hkv, B, k.stride_t, k.stride_h, k.stride_b, 128) ||
-      !make_tmap_bf16(&a.tm_v, v.ptr, d, N, Hkv, B, v.stride_t, v.stride_h, v.stride_b, 128))
+  if (!make_tmap_bf16(&a.tm_q, q.ptr, d, N_q, Hq, B, q.stride_t, q.stride_h, q.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_k, k.ptr, d, N_k, Hkv, B, k.stride_t, k.stride_h, k.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_v, v.ptr, d, N_k, Hkv, B, v.stride_t, v.stride_h, v.stride_b, 128))
     return COWA_ERR_CUDA;
   return launch_fwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
 }

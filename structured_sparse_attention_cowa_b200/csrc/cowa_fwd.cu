@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   // ---- work item: heaviest (last) query tiles first; all heads/pairs of one tile adjacent
   const int grp = a.Hq / a.Hkv;
   const int npair = (grp + 1) >> 1;
-  const int nq = (a.N + kBM - 1) / kBM;
+  const int nq = (a.Nq + kBM - 1) / kBM;
   const int per_i = a.B * a.Hkv * npair;
   const int i = nq - 1 - (int)(blockIdx.x / per_i);
   int rem = blockIdx.x % per_i;
@@ -93,7 +93,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   const int b = rem / a.Hkv;
   const int h0 = g * grp + 2 * pair;
   const bool has1 = (2 * pair + 1) < grp;
-  const int t0 = i * kBM, t1 = imin(a.N, t0 + kBM);
+  // query rows of the tile: local q rows [i*BM, ...), absolute positions [t0, t1)
+  const int t0 = a.q_off + i * kBM, t1 = imin(a.q_off + a.Nq, t0 + kBM);
   const Range iv = interval_of(a.pat, g);
   const Tiles T = plan_tiles(a.pat, iv, t0, t1);
 
@@ -133,8 +134,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       ptx::tma_prefetch_desc(&a.tm_v);
       ptx::mbar_arrive_expect_tx(&q_full, (has1 ? 2 : 1) * Geo::kQBytes);
       for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, t0, h0, b);
-        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, t0, h0 + 1, b);
+        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, i * kBM, h0, b);
+        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, i * kBM, h0 + 1, b);
       }
       TileCursor cur;
       cur.init(T);
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       cur.init(T);
       for (int n = 0; n < ntiles; ++n, cur.next(T)) {
         const int s0 = cur.j * kBN;
-        const bool need_mask = (s0 + kBN > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kBN));
+        const bool need_mask = (s0 + kBN > a.Nk) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.Nk, s0 + kBN));
         if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
         // visible key columns of row t within [s0, s0+128), relative to s0 (partial tiles only)
@@ -345,15 +346,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], 0, &abort_flag, a.status)) {
         ptx::tc_fence_after();
         const float inv = 1.f / l;
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)t * a.o_st +
+        const int rl = t - a.q_off;  // local query row
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)rl * a.o_st +
                               (size_t)(h0 + k) * a.o_sh;
-        if (t < a.N) a.lse[((size_t)b * a.Hq + h0 + k) * a.N + t] = (m_used + log2f(l)) * 0.69314718055994530942f;
+        if (t < t1) a.lse[((size_t)b * a.Hq + h0 + k) * a.Nq + rl] = (m_used + log2f(l)) * 0.69314718055994530942f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
           ptx::tmem_ld32(o_tm + c * 32, ov);  // warp-collective: every lane loads, valid rows store
           ptx::tmem_wait_ld();
-          if (t < a.N) {
+          if (t < t1) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
               uint32_t w[4];
@@ -384,7 +386,7 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
   if (e != cudaSuccess) return e;
   const int grp = a.Hq / a.Hkv;
-  const int nq = (a.N + kBM - 1) / kBM;
+  const int nq = (a.Nq + kBM - 1) / kBM;
   const long long nblk = (long long)nq * a.B * a.Hkv * ((grp + 1) / 2);
   if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
   // the in-kernel register split assumes the compiled count equals the launch allocation

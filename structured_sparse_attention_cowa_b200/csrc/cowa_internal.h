@@ -44,7 +44,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 // ---- forward ----
 struct FwdArgs {
   Pat pat;
-  int B, N, Hq, Hkv, d;
+  int B, Hq, Hkv, d;
+  int Nq, Nk, q_off;  // query rows q_off .. q_off+Nq-1 (absolute positions) against keys 0 .. Nk-1
   void* o;
   int64_t o_sb, o_st, o_sh;
   float* lse;

@@ -129,6 +129,19 @@ def test_fwd_rejects_bad_arguments_before_launch(kwargs, status):
     assert _fwd(**kwargs) == status
 
 
+@pytest.mark.parametrize("Nq,Nk,off,status", [
+    (128, 128, 1, 1),     # the block's last query position is past the keys
+    (100, 300, 201, 1),
+    (64, 64, -1, 1),      # negative offset
+    (64, 0, 0, 1),        # no keys
+    (0, 64, 0, 1),        # no queries
+])
+def test_fwd_chunk_rejects_bad_offsets_before_launch(Nq, Nk, off, status):
+    p = cw.Pattern(64, 8, 1024, 4).c()
+    assert cw.lib().cowa_fwd_chunk(ctypes.byref(p), 1, Nq, Nk, off, 8, 4, 128, _t(), _t(), _t(), _t(), 0x20000,
+                                   0x40000, 1 << 20, None) == status
+
+
 def test_decode_and_bwd_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(64, 8, 1024, 4).c()

@@ -90,6 +90,65 @@ def test_fwd_running_max_growth(cuda_device):
         assert err_o <= O_ATOL and err_l <= LSE_ATOL, (lo, hi, err_o, err_l)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_fwd_chunked_prefill(cuda_device, d):
+    """Query blocks at offsets 0, 300, 700 of a 1000-token prefill (ragged, not tile-aligned)
+    against the keys written so far: each block equals the oracle's rows and the one-pass
+    forward's rows; keys past the block (present or not) change nothing."""
+    B, N, Hq, Hkv = 1, 1000, 10, 2
+    pat = cw.Pattern(64, 128, 1000, 2)
+    q64, q = host_and_device((B, N, Hq, d), "q", cuda_device, 13)
+    k64, k = host_and_device((B, N, Hkv, d), "k", cuda_device, 13)
+    v64, v = host_and_device((B, N, Hkv, d), "v", cuda_device, 13)
+    want_o, want_l = orc.attention_fwd(q64, k64, v64, oracle_pattern(pat))
+    full_o, full_l = cw.cowa_fwd(q, k, v, pat)
+    for lo, hi, n_k in [(0, 300, 300), (300, 700, 1000), (700, 1000, 1000), (640, 1000, 1000)]:
+        o, lse = cw.cowa_fwd_chunk(q[:, lo:hi].contiguous(), k, v, pat, q_offset=lo, n_k=n_k)
+        torch.cuda.synchronize()
+        err_o = np.abs(to64(o) - want_o[:, lo:hi]).max()
+        err_l = np.abs(lse.cpu().numpy().astype(np.float64) - want_l[:, :, lo:hi]).max()
+        assert err_o <= O_ATOL and err_l <= LSE_ATOL, (lo, hi, err_o, err_l)
+        assert np.abs(to64(o) - to64(full_o[:, lo:hi])).max() <= O_ATOL
+        assert float((lse - full_l[:, :, lo:hi]).abs().max()) <= LSE_ATOL
+
+
+def test_fwd_chunked_prefill_over_a_kv_cache(cuda_device):
+    """The block's keys come from a [B, H_kv, T_cap, d] cache (as decode uses) holding the first
+    n_k positions and unrelated data after them: B=2, a 360-row block at offset 640."""
+    B, N, Hq, Hkv, d, T_cap = 2, 1000, 8, 4, 128, 1152
+    pat = cw.Pattern(32, 200, 1000, 4)
+    q64, q = host_and_device((B, N, Hq, d), "q", cuda_device, 17)
+    k64, k = host_and_device((B, N, Hkv, d), "k", cuda_device, 17)
+    v64, v = host_and_device((B, N, Hkv, d), "v", cuda_device, 17)
+    kc = synth.cuda_normal_bf16((B, Hkv, T_cap, d), 99, cuda_device)
+    vc = synth.cuda_normal_bf16((B, Hkv, T_cap, d), 98, cuda_device)
+    kc[:, :, :N] = k.transpose(1, 2)
+    vc[:, :, :N] = v.transpose(1, 2)
+    lo, hi = 640, 1000
+    o, lse = cw.cowa_fwd_chunk(q[:, lo:hi].contiguous(), kc, vc, pat, q_offset=lo, n_k=N, kv_layout="bhtd")
+    torch.cuda.synchronize()
+    want_o, want_l = orc.attention_fwd(q64, k64, v64, oracle_pattern(pat))
+    assert np.abs(to64(o) - want_o[:, lo:hi]).max() <= O_ATOL
+    assert np.abs(lse.cpu().numpy().astype(np.float64) - want_l[:, :, lo:hi]).max() <= LSE_ATOL
+
+
+def test_fwd_chunked_prefill_8k(cuda_device):
+    """Prefill 8K shapes (H_q=32, H_kv=8, S=128, L=1024, D=8): the block [4096, 6144) against
+    keys 0..6143, every row of batch 0 against the oracle."""
+    B, N, Hq, Hkv, d = 1, 8192, 32, 8, 128
+    pat = cw.Pattern(128, 1024, 8192, 8)
+    qh, q = host_and_device((B, N, Hq, d), "q", cuda_device)
+    kh, k = host_and_device((B, N, Hkv, d), "k", cuda_device)
+    vh, v = host_and_device((B, N, Hkv, d), "v", cuda_device)
+    lo, hi = 4096, 6144
+    o, lse = cw.cowa_fwd_chunk(q[:, lo:hi].contiguous(), k, v, pat, q_offset=lo, n_k=hi)
+    torch.cuda.synchronize()
+    rows = np.arange(lo, hi)
+    want_o, want_l = orc.attention_fwd_rows(qh, kh, vh, oracle_pattern(pat), rows, b=0)
+    assert np.abs(to64(o[0]) - want_o).max() <= O_ATOL
+    assert np.abs(lse[0].T.cpu().numpy().astype(np.float64) - want_l).max() <= LSE_ATOL
+
+
 def _check_fwd_rows(B, N, Hq, Hkv, d, pat, device, rows, batches, use_cuda_gen=False):
     if use_cuda_gen:
         q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), device)
