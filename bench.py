@@ -267,6 +267,7 @@ SWEEP = [  # (name, B, N, Hq, Hkv, d, S, L, T, D, bwd)
     ("prefill 8K D=2", 2, 8192, 32, 8, 128, 128, 1024, 8192, 2, False),
     ("prefill 8K D=1", 2, 8192, 32, 8, 128, 128, 1024, 8192, 1, False),
     ("train 32K dense causal", 1, 32768, 40, 8, 128, 128, 32768, 32768, 8, True),
+    ("train 32K SWA + sinks (T = S)", 1, 32768, 40, 8, 128, 128, 2048, 128, 8, True),
     ("long 128K", 1, 131072, 40, 8, 128, 128, 4096, 131072, 8, True),
     ("long 128K dense causal", 1, 131072, 40, 8, 128, 128, 131072, 131072, 8, True),
 ]
@@ -336,6 +337,21 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
     out.append({"config": "decode 128K dense causal", "B": dc["B"], "pos": dc["pos"], "decode_ms": d_ms,
                 "decode_gbs": dbytes / (d_ms * 1e-3) / 1e9, "decode_frac_hbm": dbytes / (d_ms * 1e-3) / 1e9 / hbm_gbs,
                 "bytes": dbytes})
+
+    # decode over the compacted per-head cache (sink + band ring + own interval), built from the
+    # full cache; the same visible bytes are read, the cache holds 20,736 instead of 131,072 rows
+    pat_c = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
+    kc_c, vc_c = cw.compact_cache(kc.transpose(1, 2), vc.transpose(1, 2), pat_c)
+    c_ms = timed(lambda: cw.cowa_decode_compact(qt, kc_c, vc_c, pos, pat_c, out=od))
+    toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
+    vbytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2
+    rows = cw.compact_rows(pat_c, dc["Hkv"])
+    out.append({"config": "decode 128K over the compacted cache", "B": dc["B"], "pos": dc["pos"], "decode_ms": c_ms,
+                "decode_gbs": vbytes / (c_ms * 1e-3) / 1e9, "decode_frac_hbm": vbytes / (c_ms * 1e-3) / 1e9 / hbm_gbs,
+                "cache_rows_per_head": rows, "full_cache_rows_per_head": dc["T_cap"],
+                "cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * rows * dc["d"] * 2,
+                "full_cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * dc["T_cap"] * dc["d"] * 2})
+    del kc_c, vc_c
     return out
 
 

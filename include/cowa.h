@@ -151,6 +151,38 @@ cowa_status cowa_decode(const cowa_pattern* pat, int B, int H_q, int H_kv, int d
                         const int32_t* pos, void* o, float* lse_or_null,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* ---- compacted decode cache -----------------------------------------------------------------
+ * The abstract of "CoWindow Attention: Full Causal Coverage Is a Collective Property" reports a
+ * 7.6x lower per-rank peak operator memory during decoding at 128K: a KV head never reads
+ * positions outside its sink, band and own interval, so only those need to be kept.  This layout
+ * keeps exactly that, per (b, KV head), as rows of d bf16 in one contiguous
+ * [B, H_kv, rows, d] array (rows = cowa_compact_rows):
+ *   sink       rows [0, S64)            position p < S at row p                  (S64 = S rounded up to 64)
+ *   band ring  rows [S64, S64 + R)      position p at row S64 + (p mod R)        (R = L rounded up to 64, + 64)
+ *   interval   rows [S64 + R, rows)     position p of the head's interval [lo, hi) at row
+ *                                       S64 + R + p - (lo rounded down to 64)
+ * At 128K (S=128, L=4096, T=131072, 8 KV heads) that is 20,736 rows per head instead of 131,072.
+ * The ring holds the last R positions, so positions must be appended in order (build from a
+ * prefill, then one append per decoded token).  The caller owns both arrays. */
+/* Rows per (b, KV head) of the compacted cache; 0 for an invalid pattern. */
+int cowa_compact_rows(const cowa_pattern* pat, int H_kv);
+/* Fills the compacted cache from the keys and values of positions 0..N-1 (k, v as in cowa_fwd:
+ * [B, N, H_kv, d] with any cowa_tensor strides).  Rows no position maps to are left untouched. */
+cowa_status cowa_compact_build(const cowa_pattern* pat, int B, int N, int H_kv, int d, cowa_tensor k, cowa_tensor v,
+                               void* k_compact, void* v_compact, void* stream);
+/* Appends the token at pos[b] (device int32 [B]; negative entries are skipped): k_new, v_new are
+ * [B, H_kv, d] bf16 contiguous; the token goes to every region that holds its position. */
+cowa_status cowa_compact_append(const cowa_pattern* pat, int B, int H_kv, int d, const void* k_new,
+                                const void* v_new, const int32_t* pos, void* k_compact, void* v_compact,
+                                void* stream);
+/* Decode over the compacted cache: the same result as cowa_decode over the full cache holding the
+ * same positions (pos[b] >= 0 is the new token, already appended; negative entries are clamped
+ * to 0).  Errors as for cowa_decode. */
+size_t cowa_decode_compact_workspace_size(const cowa_pattern* pat, int B, int H_q, int H_kv, int d);
+cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, const void* q_t,
+                                const void* k_compact, const void* v_compact, const int32_t* pos, void* o,
+                                float* lse_or_null, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- decode without a caller workspace -----------------------------------------------------
  * This entry point has no counterpart on the CoWA pages; it is a convenience of this library for
  * callers that cannot allocate device memory (runtimes that reserve the whole memory pool up

@@ -96,6 +96,16 @@ def lib() -> ctypes.CDLL:
     L.cowa_decode.restype = i
     L.cowa_decode_noalloc.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp]
     L.cowa_decode_noalloc.restype = i
+    L.cowa_compact_rows.argtypes = [P, i]
+    L.cowa_compact_rows.restype = i
+    L.cowa_compact_build.argtypes = [P, i, i, i, i, T, T, vp, vp, vp]
+    L.cowa_compact_build.restype = i
+    L.cowa_compact_append.argtypes = [P, i, i, i, vp, vp, vp, vp, vp, vp]
+    L.cowa_compact_append.restype = i
+    L.cowa_decode_compact_workspace_size.argtypes = [P, i, i, i, i]
+    L.cowa_decode_compact_workspace_size.restype = sz
+    L.cowa_decode_compact.argtypes = [P, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.cowa_decode_compact.restype = i
     L.cowa_workspace_status.argtypes = [vp, vp]
     L.cowa_workspace_status.restype = i
     L.cowa_status_string.argtypes = [i]
@@ -271,6 +281,74 @@ def cowa_decode(q_t, k_cache, v_cache, pos, pattern: Pattern, layout: str = "bht
                                         _cache_tensor(k_cache, layout), _cache_tensor(v_cache, layout),
                                         pos.data_ptr(), out.data_ptr(), lse.data_ptr() if lse is not None else None,
                                         workspace.data_ptr(), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def compact_rows(pattern: Pattern, h_kv: int) -> int:
+    """Rows per (b, KV head) of the compacted decode cache."""
+    n = lib().cowa_compact_rows(ctypes.byref(pattern.c()), h_kv)
+    if n <= 0:
+        raise CowaError("invalid pattern for the compacted cache")
+    return n
+
+
+def compact_cache(k, v, pattern: Pattern, out=None, stream=None):
+    """Compacted caches (k_c, v_c), [B, H_kv, rows, d] bf16, built from k, v [B, N, H_kv, d] of
+    positions 0..N-1."""
+    import torch
+
+    for n_, x_ in (("k", k), ("v", v)):
+        _bf16_cuda(n_, x_)
+    B, N, Hkv, d = k.shape
+    rows = compact_rows(pattern, Hkv)
+    if out is None:
+        out = (torch.zeros((B, Hkv, rows, d), dtype=torch.bfloat16, device=k.device),
+               torch.zeros((B, Hkv, rows, d), dtype=torch.bfloat16, device=k.device))
+    kc, vc = out
+    _check("cowa_compact_build", lib().cowa_compact_build(ctypes.byref(pattern.c()), B, N, Hkv, d, _t4(k), _t4(v),
+                                                          kc.data_ptr(), vc.data_ptr(), _stream(stream)))
+    return kc, vc
+
+
+def compact_append(kc, vc, k_new, v_new, pos, pattern: Pattern, stream=None):
+    """Appends the token at pos[b] (k_new, v_new [B, H_kv, d]) to the compacted caches in place."""
+    import torch
+
+    B, Hkv, _, d = kc.shape
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise ValueError("pos must be a CUDA int32 tensor")
+    k_new, v_new = k_new.contiguous(), v_new.contiguous()
+    _check("cowa_compact_append", lib().cowa_compact_append(ctypes.byref(pattern.c()), B, Hkv, d, k_new.data_ptr(),
+                                                            v_new.data_ptr(), pos.data_ptr(), kc.data_ptr(),
+                                                            vc.data_ptr(), _stream(stream)))
+
+
+def cowa_decode_compact(q_t, kc, vc, pos, pattern: Pattern, out=None, lse=None, workspace=None, stream=None):
+    """cowa_decode over the compacted caches kc, vc [B, H_kv, rows, d]."""
+    import torch
+
+    for n_, x_ in (("q_t", q_t), ("k_compact", kc), ("v_compact", vc)):
+        _bf16_cuda(n_, x_)
+    if not (q_t.is_contiguous() and kc.is_contiguous() and vc.is_contiguous()):
+        raise ValueError("q_t and the compacted caches must be contiguous")
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise ValueError("pos must be a CUDA int32 tensor")
+    B, Hq, d = q_t.shape
+    Hkv = kc.shape[1]
+    if kc.shape[2] != compact_rows(pattern, Hkv):
+        raise ValueError("compacted cache has the wrong number of rows for this pattern")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_t.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q_t.device)
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_decode_compact_workspace_size(ctypes.byref(pat), B, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q_t.device)
+    _check("cowa_decode_compact", L.cowa_decode_compact(ctypes.byref(pat), B, Hq, Hkv, d, q_t.data_ptr(), kc.data_ptr(),
+                                                        vc.data_ptr(), pos.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                                        workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return out, lse
 
 

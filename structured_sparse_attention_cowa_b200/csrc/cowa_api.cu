@@ -137,6 +137,83 @@ cowa_status cowa_workspace_status(void* ws, void* stream) {
 }
 
 // ------------------------------------------------------------------------------ decode
+// ------------------------------------------------------------------------------ compacted cache
+namespace {
+constexpr int kCompactSpan = 1 << 30;  // positions are unbounded: the split count follows the pattern
+}
+
+int cowa_compact_rows(const cowa_pattern* pat, int Hkv) {
+  Pat p;
+  if (Hkv < 1 || check_pattern(pat, Hkv, &p) != COWA_OK) return 0;
+  return compact_geom(p).rows;
+}
+
+cowa_status cowa_compact_build(const cowa_pattern* pat, int B, int N, int Hkv, int d, cowa_tensor k, cowa_tensor v,
+                               void* k_compact, void* v_compact, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, N, Hkv, Hkv, d));
+  COWA_TRY(check_tensor(k));
+  COWA_TRY(check_tensor(v));
+  if (!k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(k_compact) || !aligned16(v_compact)) return COWA_ERR_ALIGNMENT;
+  return launch_compact_build(p, B, N, Hkv, d, k.ptr, k.stride_b, k.stride_t, k.stride_h, v.ptr, v.stride_b,
+                              v.stride_t, v.stride_h, k_compact, v_compact,
+                              reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
+}
+
+cowa_status cowa_compact_append(const cowa_pattern* pat, int B, int Hkv, int d, const void* k_new, const void* v_new,
+                                const int32_t* pos, void* k_compact, void* v_compact, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, 1, Hkv, Hkv, d));
+  if (!k_new || !v_new || !pos || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_compact) || !aligned16(v_compact))
+    return COWA_ERR_ALIGNMENT;
+  return launch_compact_append(p, B, Hkv, d, k_new, v_new, pos, k_compact, v_compact,
+                               reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
+}
+
+size_t cowa_decode_compact_workspace_size(const cowa_pattern* pat, int B, int Hq, int Hkv, int d) {
+  return cowa_decode_workspace_size(pat, B, Hq, Hkv, d, kCompactSpan);
+}
+
+cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, const void* q_t,
+                                const void* k_compact, const void* v_compact, const int32_t* pos, void* o,
+                                float* lse_or_null, void* ws, size_t ws_bytes, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, 1, Hq, Hkv, d));
+  if (!q_t || !pos || !o || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(q_t) || !aligned16(o) || !aligned16(k_compact) || !aligned16(v_compact) ||
+      (lse_or_null && (reinterpret_cast<uintptr_t>(lse_or_null) & 3u)))
+    return COWA_ERR_ALIGNMENT;
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_decode_compact_workspace_size(pat, B, Hq, Hkv, d)));
+
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.pat = p; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.T_cap = kCompactSpan;
+  a.q_t = q_t; a.pos = pos; a.o = o; a.lse = lse_or_null;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.chunk = decode_chunk_tokens(p, B, Hkv, kCompactSpan);
+  a.n_split = decode_num_splits(p, kCompactSpan, a.chunk);
+  a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f;
+  a.compact = 1;
+  a.cg = compact_geom(p);
+  const int64_t rows = a.cg.rows;
+  if (!make_tmap_bf16(&a.tm_k, k_compact, d, (int)rows, Hkv, B, d, rows * d, (int64_t)Hkv * rows * d,
+                      64) ||
+      !make_tmap_bf16(&a.tm_v, v_compact, d, (int)rows, Hkv, B, d, rows * d, (int64_t)Hkv * rows * d,
+                      64))
+    return COWA_ERR_CUDA;
+  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+}
+
 size_t cowa_decode_workspace_size(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, int T_cap) {
   Pat p;
   if (check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(B, 1, Hq, Hkv, d) != COWA_OK || T_cap < 1) return 0;

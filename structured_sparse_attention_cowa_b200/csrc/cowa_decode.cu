@@ -69,24 +69,51 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 
   // ---- which chunk of which visible range this CTA owns (pure position arithmetic)
   int t = a.pos[b];
-  t = t < 0 ? 0 : (t >= a.T_cap ? a.T_cap - 1 : t);
+  t = t < 0 ? 0 : (a.compact || t < a.T_cap ? t : a.T_cap - 1);
   const Range iv = interval_of(a.pat, g);
   Range rr[3];
-  const int nr = row_ranges(a.pat, iv, t, rr);
-  int c_lo = 0, c_hi = 0;
+  int region[3] = {0, 0, 0};
+  int nr;
+  if (!a.compact) {
+    nr = row_ranges(a.pat, iv, t, rr);  // merged ranges of positions = cache rows
+  } else {
+    // three disjoint sets, each read from its own region: sink, the interval keys before the
+    // band, the band without the sink
+    const int sink_hi = imin(a.pat.S, t + 1);
+    const int band_lo = imax(0, t - a.pat.L + 1);
+    rr[0] = Range{0, sink_hi};
+    rr[1] = Range{iv.lo, imin(imin(iv.hi, t + 1), band_lo)};
+    rr[2] = Range{imax(band_lo, sink_hi), t + 1};
+    region[0] = 0; region[1] = 1; region[2] = 2;
+    nr = 3;
+  }
+  int c_lo = 0, c_hi = 0, c_reg = 0;
   {
     int idx = split;
     for (int r = 0; r < nr; ++r) {
-      const int nch = (rr[r].hi - rr[r].lo + a.chunk - 1) / a.chunk;
+      const int len = rr[r].hi - rr[r].lo;
+      const int nch = len > 0 ? (len + a.chunk - 1) / a.chunk : 0;
       if (idx < nch) {
         c_lo = rr[r].lo + idx * a.chunk;
         c_hi = imin(rr[r].hi, c_lo + a.chunk);
+        c_reg = region[r];
         break;
       }
       idx -= nch;
     }
   }
-  const int nsub = (c_hi - c_lo + kSubTok - 1) / kSubTok;
+  // sub-tiles start at c_lo (full cache) or at the 64-aligned position below it (compacted
+  // cache: an aligned block is 64 consecutive rows of one region); tokens outside
+  // [c_lo, c_hi) are masked
+  const int p_base = a.compact ? (c_lo & ~(kSubTok - 1)) : c_lo;
+  const int nsub = c_hi > c_lo ? (c_hi - p_base + kSubTok - 1) / kSubTok : 0;
+  const int lo64 = iv.lo & ~(kSubTok - 1);
+  auto cache_row = [&](int pp) -> int {  // cache row of the sub-tile at position pp
+    if (!a.compact) return pp;
+    if (c_reg == 0) return pp;
+    if (c_reg == 1) return a.cg.IB + (pp - lo64);
+    return a.cg.S64 + (pp % a.cg.R);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -111,11 +138,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         uint8_t* ks = smem + s * Geo::kStageBytes;
         uint8_t* vs = ks + Geo::kTileBytes;
         ptx::mbar_arrive_expect_tx(&full_bar[s], Geo::kStageBytes);
-        const int t0 = c_lo + st * kSubTok;
+        const int row = cache_row(p_base + st * kSubTok);
 #pragma unroll
         for (int u = 0; u < Geo::kUnits; ++u) {
-          ptx::tma_load_4d(ks + u * kBoxBytes, &a.tm_k, &full_bar[s], u * 64, t0, g, b);
-          ptx::tma_load_4d(vs + u * kBoxBytes, &a.tm_v, &full_bar[s], u * 64, t0, g, b);
+          ptx::tma_load_4d(ks + u * kBoxBytes, &a.tm_k, &full_bar[s], u * 64, row, g, b);
+          ptx::tma_load_4d(vs + u * kBoxBytes, &a.tm_v, &full_bar[s], u * 64, row, g, b);
         }
         issued = st + 1;
       }
@@ -169,12 +196,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
       }
     }
     // ---- online softmax (log2 domain) over this warp's 16 tokens
-    const int tok0 = c_lo + st * kSubTok + row0 + 2 * tq;
+    const int tok0 = p_base + st * kSubTok + row0 + 2 * tq;
     float x[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int tok = tok0 + 8 * (e >> 1) + (e & 1);
-      x[e] = tok < c_hi ? sc[e >> 1][e & 1] * a.scale_log2 : -INFINITY;
+      x[e] = (tok >= c_lo && tok < c_hi) ? sc[e >> 1][e & 1] * a.scale_log2 : -INFINITY;
     }
     float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -276,6 +303,58 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const __grid_consta
   if (a.lse && lane == 0) a.lse[wid] = (mx + log2f(l)) * 0.69314718055994530942f;
 }
 
+// ------------------------------------------------------------------ compacted cache upkeep
+// Appends the token at pos[b] (k_new / v_new [B, H_kv, D] contiguous) to every region that holds
+// it.  One block per (KV head, b); 16-byte copies.
+template <int D>
+__global__ void __launch_bounds__(D / 8) compact_append_kernel(Pat pat, CompactGeom cg, const uint4* k_new,
+                                                                 const uint4* v_new, const int32_t* pos, uint4* kc,
+                                                                 uint4* vc, int Hkv) {
+  const int g = blockIdx.x, b = blockIdx.y, u = threadIdx.x;
+  const int p = pos[b];
+  if (p < 0) return;
+  const Range iv = interval_of(pat, g);
+  const size_t src = ((size_t)b * Hkv + g) * (D / 8) + u;
+  const uint4 kk = k_new[src], vv = v_new[src];
+  const size_t head = ((size_t)b * Hkv + g) * (size_t)cg.rows;
+  auto put = [&](int row) {
+    kc[(head + row) * (D / 8) + u] = kk;
+    vc[(head + row) * (D / 8) + u] = vv;
+  };
+  put(cg.S64 + p % cg.R);
+  if (p < pat.S) put(p);
+  if (p >= iv.lo && p < iv.hi) put(cg.IB + p - (iv.lo & ~(kSubTok - 1)));
+}
+
+// Builds the compacted cache from the keys and values of positions 0..N-1 (strided
+// [B, N, H_kv, D]): block (x, g, b) handles positions [64x, 64x + 64).
+template <int D>
+__global__ void __launch_bounds__(128) compact_build_kernel(Pat pat, CompactGeom cg, const __nv_bfloat16* k,
+                                                             const __nv_bfloat16* v, int64_t sb, int64_t st,
+                                                             int64_t sh, int64_t vsb, int64_t vst, int64_t vsh,
+                                                             int N, uint4* kc, uint4* vc, int Hkv) {
+  const int g = blockIdx.y, b = blockIdx.z;
+  const Range iv = interval_of(pat, g);
+  const int lo64 = iv.lo & ~(kSubTok - 1);
+  const size_t head = ((size_t)b * Hkv + g) * (size_t)cg.rows;
+  constexpr int U = D / 8;
+  for (int x = threadIdx.x; x < kSubTok * U; x += blockDim.x) {
+    const int p = blockIdx.x * kSubTok + x / U, u = x % U;
+    if (p >= N) continue;
+    const bool in_ring = p >= N - cg.R, in_sink = p < pat.S, in_iv = p >= iv.lo && p < iv.hi;
+    if (!in_ring && !in_sink && !in_iv) continue;
+    const uint4 kk = reinterpret_cast<const uint4*>(k + b * sb + (int64_t)p * st + g * sh)[u];
+    const uint4 vv = reinterpret_cast<const uint4*>(v + b * vsb + (int64_t)p * vst + g * vsh)[u];
+    auto put = [&](int row) {
+      kc[(head + row) * U + u] = kk;
+      vc[(head + row) * U + u] = vv;
+    };
+    if (in_ring) put(cg.S64 + p % cg.R);
+    if (in_sink) put(p);
+    if (in_iv) put(cg.IB + p - lo64);
+  }
+}
+
 template <int GRP, int D>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
   using Geo = DecGeom<D>;
@@ -322,6 +401,56 @@ int decode_num_splits(const Pat& p, int T_cap, int chunk) {
   const int64_t lr = wmax < T_cap ? wmax : T_cap;
   int64_t n = (sink + chunk - 1) / chunk + (lr + chunk - 1) / chunk + (band + chunk - 1) / chunk;
   return (int)(n < 1 ? 1 : n);
+}
+
+CompactGeom compact_geom(const Pat& p) {
+  CompactGeom c;
+  c.S64 = (p.S + kSubTok - 1) / kSubTok * kSubTok;
+  c.R = (p.L + kSubTok - 1) / kSubTok * kSubTok + kSubTok;
+  c.IB = c.S64 + c.R;
+  int w = 0;
+  for (int slot = 0; slot < p.H; slot += p.H / p.D) {  // the distinct interval slots
+    const int lo = bound(p, slot), hi = bound(p, slot + 1);
+    if (hi > lo) w = imax(w, hi - (lo & ~(kSubTok - 1)));
+  }
+  c.W = (w + kSubTok - 1) / kSubTok * kSubTok;
+  c.rows = c.IB + c.W;
+  return c;
+}
+
+cudaError_t launch_compact_append(const Pat& p, int B, int Hkv, int d, const void* k_new, const void* v_new,
+                                  const int32_t* pos, void* kc, void* vc, cudaStream_t s) {
+  const CompactGeom cg = compact_geom(p);
+  dim3 grid(Hkv, B);
+  if (d == 128)
+    compact_append_kernel<128><<<grid, 16, 0, s>>>(p, cg, static_cast<const uint4*>(k_new),
+                                                   static_cast<const uint4*>(v_new), pos, static_cast<uint4*>(kc),
+                                                   static_cast<uint4*>(vc), Hkv);
+  else if (d == 64)
+    compact_append_kernel<64><<<grid, 8, 0, s>>>(p, cg, static_cast<const uint4*>(k_new),
+                                                 static_cast<const uint4*>(v_new), pos, static_cast<uint4*>(kc),
+                                                 static_cast<uint4*>(vc), Hkv);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact_build(const Pat& p, int B, int N, int Hkv, int d, const void* k, int64_t ksb, int64_t kst,
+                                 int64_t ksh, const void* v, int64_t vsb, int64_t vst, int64_t vsh, void* kc, void* vc,
+                                 cudaStream_t s) {
+  const CompactGeom cg = compact_geom(p);
+  dim3 grid((N + kSubTok - 1) / kSubTok, Hkv, B);
+  auto kb = static_cast<const __nv_bfloat16*>(k);
+  auto vb = static_cast<const __nv_bfloat16*>(v);
+  if (d == 128)
+    compact_build_kernel<128><<<grid, 128, 0, s>>>(p, cg, kb, vb, ksb, kst, ksh, vsb, vst, vsh, N,
+                                                   static_cast<uint4*>(kc), static_cast<uint4*>(vc), Hkv);
+  else if (d == 64)
+    compact_build_kernel<64><<<grid, 128, 0, s>>>(p, cg, kb, vb, ksb, kst, ksh, vsb, vst, vsh, N,
+                                                  static_cast<uint4*>(kc), static_cast<uint4*>(vc), Hkv);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {

@@ -23,6 +23,17 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n_t, int n_h,
                     int64_t stride_h, int64_t stride_b, int box_rows);
 
 // ---- decode ----
+// Compacted per-head decode cache: only what decode can see, rows of d bf16 per (b, KV head):
+//   sink      rows [0, S64)           position p < S at row p
+//   band ring rows [S64, S64 + R)     position p at row S64 + (p mod R); R = round64(L) + 64
+//   interval  rows [IB, IB + W)       position p of the head's interval [lo, hi) at row
+//                                     IB + p - round_down64(lo); IB = S64 + R
+// Every 64-aligned block of positions maps to 64 consecutive rows of one region.
+struct CompactGeom {
+  int S64, R, IB, W, rows;
+};
+CompactGeom compact_geom(const Pat& p);
+
 struct DecodeArgs {
   Pat pat;
   int B, Hq, Hkv, d, T_cap;
@@ -35,11 +46,19 @@ struct DecodeArgs {
   int chunk;         // tokens per split
   int n_split;
   float scale_log2;  // softmax scale * log2(e)
+  // compacted cache (tm_k / tm_v over [B, H_kv, rows, d]): 0 = full cache indexed by position
+  int compact;
+  CompactGeom cg;
   CUtensorMap tm_k, tm_v;
 };
 int decode_chunk_tokens(const Pat& p, int B, int Hkv, int T_cap);
 int decode_num_splits(const Pat& p, int T_cap, int chunk);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_compact_append(const Pat& p, int B, int Hkv, int d, const void* k_new, const void* v_new,
+                                  const int32_t* pos, void* kc, void* vc, cudaStream_t s);
+cudaError_t launch_compact_build(const Pat& p, int B, int N, int Hkv, int d, const void* k, int64_t ksb, int64_t kst,
+                                 int64_t ksh, const void* v, int64_t vsb, int64_t vst, int64_t vsh, void* kc, void* vc,
+                                 cudaStream_t s);
 
 // ---- forward ----
 struct FwdArgs {

@@ -142,6 +142,44 @@ def test_fwd_chunk_rejects_bad_offsets_before_launch(Nq, Nk, off, status):
                                    0x40000, 1 << 20, None) == status
 
 
+@pytest.mark.parametrize("pat,Hkv", [
+    (cw.Pattern(128, 4096, 131072, 8), 8),
+    (cw.Pattern(20, 100, 2000, 2), 2),
+    (cw.Pattern(0, 70, 1800, 4), 4),
+    (cw.Pattern(64, 256, 1500, 1), 2),
+    (cw.Pattern(16, 90, 16, 2), 2),
+    (cw.Pattern(3, 9, 257, 2, kv_head_base=2, h_kv_global=4), 2),
+])
+def test_compact_cache_rows_hold_every_visible_position(pat, Hkv):
+    """The compacted layout has room for what decode can see at any position: the sink, the
+    band rounded out to 64-aligned blocks, and each head's interval from its 64-aligned start;
+    at 128K it is 20,736 rows per head (6.3x fewer than the 131,072 of the full cache)."""
+    rows = cw.lib().cowa_compact_rows(ctypes.byref(pat.c()), Hkv)
+    H = pat.h_kv_global or Hkv
+    b = orc.interval_bounds(pat.S, pat.T, H)
+    up = lambda x: -(-x // 64) * 64
+    slots = range(0, H, H // pat.D)  # the D distinct interval slots (G mod D) * (H / D)
+    need_iv = max([b[j + 1] - b[j] // 64 * 64 for j in slots if b[j + 1] > b[j]], default=0)
+    # every 64-aligned block of the band (at most L + 63 positions back from t) fits the ring
+    assert rows >= up(pat.S) + up(pat.L + 63) + up(need_iv)
+    assert rows <= up(pat.S) + up(pat.L) + 64 + up(need_iv)
+    if (pat.S, pat.L, pat.T, pat.D) == (128, 4096, 131072, 8):
+        assert rows == 20736
+
+
+def test_compact_entry_points_reject_bad_arguments():
+    L = cw.lib()
+    p = cw.Pattern(20, 100, 2000, 2).c()
+    assert L.cowa_compact_rows(None, 2) == 0
+    assert L.cowa_compact_append(ctypes.byref(p), 2, 2, 128, 0x10000, 0x20000, None, 0x30000, 0x40000, None) == 1
+    assert L.cowa_compact_append(ctypes.byref(p), 2, 2, 96, 0x10000, 0x20000, 0x50000, 0x30000, 0x40000, None) == 2
+    assert L.cowa_compact_build(ctypes.byref(p), 2, 100, 2, 128, _t(), _t(), 0x30008, 0x40000, None) == 3
+    n = L.cowa_decode_compact_workspace_size(ctypes.byref(p), 2, 8, 2, 128)
+    assert n > 256
+    assert L.cowa_decode_compact(ctypes.byref(p), 2, 8, 2, 128, 0x10000, 0x30000, 0x40000, 0x50000, 0x60000, None,
+                                 0x70000, n - 1, None) == 4
+
+
 def test_decode_and_bwd_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(64, 8, 1024, 4).c()
