@@ -179,7 +179,11 @@ cowa_status cowa_compact_append(const cowa_pattern* pat, int B, int Hkv, int d, 
 }
 
 size_t cowa_decode_compact_workspace_size(const cowa_pattern* pat, int B, int Hq, int Hkv, int d) {
-  return cowa_decode_workspace_size(pat, B, Hq, Hkv, d, kCompactSpan);
+  Pat p;
+  if (check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(B, 1, Hq, Hkv, d) != COWA_OK) return 0;
+  const int chunk = decode_chunk_tokens(p, B, Hkv, kCompactSpan);
+  const int ns = decode_num_splits(p, kCompactSpan, chunk, true);
+  return kWsHeader + align_up((size_t)B * Hq * ns * (d + 2) * sizeof(float), 256);
 }
 
 cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, const void* q_t,
@@ -201,7 +205,7 @@ cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int Hq, int Hkv,
   a.status = reinterpret_cast<uint32_t*>(ws);
   a.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
   a.chunk = decode_chunk_tokens(p, B, Hkv, kCompactSpan);
-  a.n_split = decode_num_splits(p, kCompactSpan, a.chunk);
+  a.n_split = decode_num_splits(p, kCompactSpan, a.chunk, true);
   a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f;
   a.compact = 1;
   a.cg = compact_geom(p);

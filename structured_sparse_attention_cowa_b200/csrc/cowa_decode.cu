@@ -87,15 +87,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     region[0] = 0; region[1] = 1; region[2] = 2;
     nr = 3;
   }
+  // chunks of each range: cut from its start on the full cache; on the compacted cache cut at
+  // 64-aligned positions (chunk is a multiple of 64), so only a range's first chunk begins
+  // inside a 64-row block
   int c_lo = 0, c_hi = 0, c_reg = 0;
   {
     int idx = split;
     for (int r = 0; r < nr; ++r) {
-      const int len = rr[r].hi - rr[r].lo;
-      const int nch = len > 0 ? (len + a.chunk - 1) / a.chunk : 0;
+      if (rr[r].hi <= rr[r].lo) continue;
+      const int base = a.compact ? (rr[r].lo & ~(kSubTok - 1)) : rr[r].lo;
+      const int nch = (rr[r].hi - base + a.chunk - 1) / a.chunk;
       if (idx < nch) {
-        c_lo = rr[r].lo + idx * a.chunk;
-        c_hi = imin(rr[r].hi, c_lo + a.chunk);
+        c_lo = imax(rr[r].lo, base + idx * a.chunk);
+        c_hi = imin(rr[r].hi, base + (idx + 1) * a.chunk);
         c_reg = region[r];
         break;
       }
@@ -392,14 +396,16 @@ int decode_chunk_tokens(const Pat& p, int B, int Hkv, int T_cap) {
   return 1024;
 }
 
-int decode_num_splits(const Pat& p, int T_cap, int chunk) {
-  // chunks of the three ranges, each cut from its own start: sink, widest interval, band
+int decode_num_splits(const Pat& p, int T_cap, int chunk, bool compact) {
+  // chunks of the three ranges, each cut from its own start (compacted cache: from the
+  // 64-aligned position below it, up to 63 more positions per range): sink, widest interval, band
   const int64_t R = (int64_t)p.T - p.S;
   const int64_t wmax = R > 0 ? (R + p.H - 1) / p.H : 0;
   const int64_t sink = p.S < T_cap ? p.S : T_cap;
   const int64_t band = p.L < T_cap ? p.L : T_cap;
   const int64_t lr = wmax < T_cap ? wmax : T_cap;
-  int64_t n = (sink + chunk - 1) / chunk + (lr + chunk - 1) / chunk + (band + chunk - 1) / chunk;
+  const int64_t a = compact ? kSubTok - 1 : 0;
+  int64_t n = (sink + a + chunk - 1) / chunk + (lr + a + chunk - 1) / chunk + (band + a + chunk - 1) / chunk;
   return (int)(n < 1 ? 1 : n);
 }
 

@@ -52,7 +52,7 @@ struct DecodeArgs {
   CUtensorMap tm_k, tm_v;
 };
 int decode_chunk_tokens(const Pat& p, int B, int Hkv, int T_cap);
-int decode_num_splits(const Pat& p, int T_cap, int chunk);
+int decode_num_splits(const Pat& p, int T_cap, int chunk, bool compact = false);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_compact_append(const Pat& p, int B, int Hkv, int d, const void* k_new, const void* v_new,
                                   const int32_t* pos, void* kc, void* vc, cudaStream_t s);
