@@ -345,9 +345,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
 
 // ------------------------------------------------------------------------------ dQ
 // TMEM columns: S [0,128), dP [128,256), dQ [256, 256+D), dS double buffer 2 x 64 after dQ.
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
+// NP softmax warps per TMEM lane quadrant (each owns 128/NP key columns of S and dP and D/NP
+// columns of the dQ accumulator), then the TMA producer and the MMA issuer.
+template <int D, int NP>
+__global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __grid_constant__ BwdArgs a) {
   using Geo = BwdGeom<D>;
+  constexpr int kSoftWarps = 4 * NP, kQProducer = 4 * NP, kQMma = 4 * NP + 1;
+  constexpr int CW = kTile / NP;  // key columns per softmax warp
   constexpr uint32_t kColDS = Geo::kColAcc + D;  // first dS buffer
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -383,16 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     for (int s = 0; s < KS; ++s) { ptx::mbar_init(&k_full[s], 1); ptx::mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < VS; ++s) { ptx::mbar_init(&v_full[s], 1); ptx::mbar_init(&v_empty[s], 1); }
     ptx::mbar_init(&sdp_full, 1);
-    ptx::mbar_init(&consumed_s, kComputeWarps);
-    ptx::mbar_init(&consumed_dp, kComputeWarps);
-    ptx::mbar_init(&ds_ready[0], kComputeWarps);
-    ptx::mbar_init(&ds_ready[1], kComputeWarps);
+    ptx::mbar_init(&consumed_s, kSoftWarps);
+    ptx::mbar_init(&consumed_dp, kSoftWarps);
+    ptx::mbar_init(&ds_ready[0], kSoftWarps);
+    ptx::mbar_init(&ds_ready[1], kSoftWarps);
     ptx::mbar_init(&acc_full, 1);
     ptx::mbar_init(&mma_final, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kQMma) {
     ptx::tmem_alloc(&tmem_base_sh, 512);
     ptx::tmem_relinquish();
   }
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == kProducerWarp) {
+  if (warp == kQProducer) {
     if (lane == 0) {
       ptx::tma_prefetch_desc(&a.tm_k);
       ptx::tma_prefetch_desc(&a.tm_v);
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       for (int n = (nk > KS ? nk - KS : 0); n < nk; ++n) ptx::mbar_wait(&k_full[n % KS], (n / KS) & 1, nullptr, a.status);
       for (int n = (nv > VS ? nv - VS : 0); n < nv; ++n) ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, nullptr, a.status);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kQMma) {
     // whole warp on the issue path, one elected lane issues (uniform descriptors)
     constexpr uint32_t idesc_s = ptx::idesc_bf16(128, 128, false, false);
     constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
     __syncwarp();
   } else {
-    const int quad = warp & 3, half = warp >> 2;
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;  // query row = TMEM lane
     const int t = t0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -508,12 +512,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       const bool need_mask = (s0 + kTile > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kTile));
       if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
-      uint32_t sv[64], pv[64];
-      ptx::tmem_ld32(lane_base + half * 64, sv);
-      ptx::tmem_ld32(lane_base + half * 64 + 32, sv + 32);
+      uint32_t sv[CW], pv[CW];
+#pragma unroll
+      for (int c = 0; c < CW / 32; ++c) ptx::tmem_ld32(lane_base + part * CW + 32 * c, sv + 32 * c);
       ptx::tmem_wait_ld();
-      ptx::tmem_ld32(lane_base + 128 + half * 64, pv);  // in flight while S is released
-      ptx::tmem_ld32(lane_base + 128 + half * 64 + 32, pv + 32);
+#pragma unroll
+      for (int c = 0; c < CW / 32; ++c)  // in flight while S is released
+        ptx::tmem_ld32(lane_base + 128 + part * CW + 32 * c, pv + 32 * c);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&consumed_s);  // S columns may be overwritten now
@@ -527,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       auto chunks = [&](auto masked) {
         constexpr bool kMask = decltype(masked)::value;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < CW / 32; ++c) {
           uint32_t dw[16];
 #pragma unroll
           for (int c2 = 0; c2 < 16; ++c2) {
@@ -538,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
               const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lse2);
               float p = (!kMask && use_poly && poly_col<COWA_DQ_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
               if (kMask) {
-                const int s = s0 + half * 64 + cl;
+                const int s = s0 + part * CW + cl;
                 const bool vis = s <= t && (s < sink_end || s >= band_lo || (s >= lr_lo && s < lr_hi));
                 if (!vis) p = 0.f;
               }
@@ -546,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
             }
             dw[c2] = ptx::pack_bf16(d2[0], d2[1]);
           }
-          ptx::tmem_st16(lane_base + kColDS + (n & 1) * 64 + half * 32 + 16 * c, dw);
+          ptx::tmem_st16(lane_base + kColDS + (n & 1) * 64 + part * (CW / 2) + 16 * c, dw);
         }
       };
       if (need_mask) chunks(std::true_type{});
@@ -558,14 +563,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
     }
     if (ok && ntiles > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
       ptx::tc_fence_after();
-      constexpr int HC = D / 2;
+      constexpr int HC = D / NP;  // accumulator columns of this warp
+      static_assert(HC % 32 == 0, "dQ columns per softmax warp must be whole 32-column loads");
       uint32_t dqv[HC];
 #pragma unroll
-      for (int c = 0; c < HC / 32; ++c) ptx::tmem_ld32(lane_base + Geo::kColAcc + half * HC + c * 32, dqv + c * 32);
+      for (int c = 0; c < HC / 32; ++c) ptx::tmem_ld32(lane_base + Geo::kColAcc + part * HC + c * 32, dqv + c * 32);
       ptx::tmem_wait_ld();
       if (t < a.N) {
         __nv_bfloat16* dqr = reinterpret_cast<__nv_bfloat16*>(a.dq) + b * a.dq_sb + (int64_t)t * a.dq_st +
-                             h * a.dq_sh + half * HC;
+                             h * a.dq_sh + part * HC;
 #pragma unroll
         for (int c8 = 0; c8 < HC / 8; ++c8) {
           uint32_t w[4];
@@ -581,11 +587,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kQMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
 }
+
+// softmax warps per lane quadrant of the dQ kernel: 4 at d = 128 (32 key columns each); at d = 64
+// the accumulator's 64 columns allow 2
+#ifndef COWA_DQ_PARTS
+#define COWA_DQ_PARTS 4
+#endif
+template <int D>
+constexpr int kDqParts = D == 128 ? COWA_DQ_PARTS : 2;
 
 template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
@@ -606,12 +620,13 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (stages & COWA_BWD_DQ) {
-    auto kdq = bwd_dq_kernel<D>;
+    constexpr int NP = kDqParts<D>;
+    auto kdq = bwd_dq_kernel<D, NP>;
     if ((e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemQ)) != cudaSuccess)
       return e;
     const long long n_q = (long long)nq * a.Hq * a.B;
     if (n_q > 0x7fffffffLL) return cudaErrorInvalidValue;
-    kdq<<<(unsigned)n_q, kThreads, Geo::kSmemQ, s>>>(a);
+    kdq<<<(unsigned)n_q, (4 * NP + 2) * 32, Geo::kSmemQ, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
