@@ -22,8 +22,9 @@
 //      softmax warps load S and dP of a KV tile into registers and release them at once, so
 //      the MMA warp computes S and dP of the next tile while dS of this one is being formed;
 //      dS goes to a double-buffered bf16 region of TMEM and dQ += dS K reads it as A.
-// Warp roles in both attention kernels: warps 0-7 elementwise softmax (two warps per TMEM
-// lane quadrant, each owning half of the columns), warp 8 TMA producer, warp 9 MMA issuer.
+// Warp roles in both attention kernels: 4 NP elementwise softmax warps (NP per TMEM lane
+// quadrant, each owning 1/NP of the columns; dQ: NP = 4 at d = 128, dK/dV: NP = 2), then the
+// TMA producer and the MMA issuer.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -37,9 +38,6 @@
 namespace cowa {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kComputeWarps = 8;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kStatBytes = 1024;  // lse2[128] + delta[128] of one query tile
 
 // Which exponentials run on the FMA pipe (exp2_poly.cuh) instead of the special-function unit:
@@ -103,13 +101,22 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_consta
 
 // ------------------------------------------------------------------------------ dK / dV
 // TMEM columns: two sub-step buffers at 0 and 128, each S^T [+0, +64) and dP^T [+64, +128)
-// for 64 query rows; dV [256, 256+D), dK [256+D, 256+2D).  The packed bf16 P^T and dS^T of a
-// buffer (32 columns each) start at +kColPT / +kColDST.
-constexpr uint32_t kColPT = 16, kColDST = 80;
+// for 64 query rows; dV [256, 256+D), dK [256+D, 256+2D).  NP softmax warps per lane quadrant
+// each own CW = 64/NP query columns; a warp writes its packed bf16 P^T (dS^T) into the upper
+// half of the S^T (dP^T) columns it has just read, so no warp overwrites columns another warp
+// has yet to read.  K step kk (16 query rows) of the dV / dK MMAs reads A at pt_col(kk) and
+// 64 + pt_col(kk).
 constexpr int kSub = 64;  // query rows per sub-step
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
+template <int NP>
+__device__ __forceinline__ constexpr uint32_t pt_col(int kk) {
+  constexpr int CW = kSub / NP, KPW = CW / 16;  // query columns and K steps per warp
+  return (uint32_t)((kk / KPW) * CW + CW / 2 + 8 * (kk % KPW));
+}
+template <int D, int NP>
+__global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __grid_constant__ BwdArgs a) {
   using Geo = BwdGeom<D>;
+  constexpr int kSoftWarps = 4 * NP, kKProducer = 4 * NP, kKMma = 4 * NP + 1;
+  constexpr int CW = kSub / NP;  // query columns per softmax warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   __shared__ __align__(8) uint64_t kv_full, slot_full[2], slot_empty[2], sdp_full[2], p_ready[2], acc_full,
@@ -138,14 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     for (int s = 0; s < 2; ++s) { ptx::mbar_init(&slot_full[s], 1); ptx::mbar_init(&slot_empty[s], 1); }
     for (int bb = 0; bb < 2; ++bb) {
       ptx::mbar_init(&sdp_full[bb], 1);
-      ptx::mbar_init(&p_ready[bb], kComputeWarps);
+      ptx::mbar_init(&p_ready[bb], kSoftWarps);
     }
     ptx::mbar_init(&acc_full, 1);
     ptx::mbar_init(&mma_final, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kKMma) {
     ptx::tmem_alloc(&tmem_base_sh, 512);
     ptx::tmem_relinquish();
   }
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
   const uint32_t tmem = tmem_base_sh;
   const int nsub = 2 * nsteps;  // 64-row sub-steps
 
-  if (warp == kProducerWarp) {
+  if (warp == kKProducer) {
     if (lane == 0) {
       ptx::tma_prefetch_desc(&a.tm_q);
       ptx::tma_prefetch_desc(&a.tm_do);
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
         ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, nullptr, a.status);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kKMma) {
     // whole warp on the issue path, one elected lane issues (uniform descriptors)
     constexpr uint32_t idesc_s = ptx::idesc_bf16(128, kSub, false, false);
     constexpr uint32_t idesc_o = ptx::idesc_bf16(128, D, false, true);
@@ -228,11 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       // dV += P^T dO  and  dK += dS^T Q : A (P^T, dS^T) in TMEM, B (dO, Q) MN-major in smem
 #pragma unroll
       for (int kk = 0; kk < kSub / 16; ++kk)
-        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc, buf + kColPT + kk * 8,
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc, buf + pt_col<NP>(kk),
                               ptx::desc_advance(slot_desc_mn, do_off + kk * 2048), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < kSub / 16; ++kk)
-        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc + D, buf + kColDST + kk * 8,
+        ptx::mma_bf16_ts_warp(tmem + Geo::kColAcc + D, buf + 64 + pt_col<NP>(kk),
                               ptx::desc_advance(slot_desc_mn, q_off + kk * 2048), idesc_o, (m > 0 || kk > 0) ? 1u : 0u);
       if (hq == 1) ptx::mma_commit_warp(&slot_empty[n & 1]);
     }
@@ -241,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     ptx::mbar_wait(&mma_final, 0, nullptr, a.status);
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ elementwise softmax (8 warps)
-    const int quad = warp & 3, half = warp >> 2;
+    // ------------------------------------------------------------ elementwise softmax (4 NP warps)
+    const int quad = warp & 3, part = warp >> 2;
     const int r = quad * 32 + lane;  // key row of the tile = TMEM lane
     const int s = s0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -257,22 +264,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
       if (!(ok = ptx::mbar_wait_warp(&sdp_full[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
       const uint32_t buf = lane_base + 128 * (m & 1);
-      // this warp's 32 query columns of the sub-step
-      uint32_t sv[32], pv[32];
-      ptx::tmem_ld32(buf + 32 * half, sv);
-      ptx::tmem_ld32(buf + 64 + 32 * half, pv);
+      // this warp's CW query columns of the sub-step
+      uint32_t sv[CW], pv[CW];
+      if constexpr (CW == 32) {
+        ptx::tmem_ld32(buf + CW * part, sv);
+        ptx::tmem_ld32(buf + 64 + CW * part, pv);
+      } else {
+        ptx::tmem_ld16(buf + CW * part, sv);
+        ptx::tmem_ld16(buf + 64 + CW * part, pv);
+      }
       ptx::tmem_wait_ld();
       const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes) +
-                          hq * kSub + 32 * half;
+                          hq * kSub + CW * part;
       const bool use_poly = !need_mask && t0 + kSub <= a.N;
       // the element loop is instantiated with and without the mask, chosen once per sub-step
       auto body = [&](auto masked) {
         constexpr bool kMask = decltype(masked)::value;
         const float4* lse4 = reinterpret_cast<const float4*>(stat);
         const float4* del4 = reinterpret_cast<const float4*>(stat + 128);
-        uint32_t pw[16], dw[16];
+        uint32_t pw[CW / 2], dw[CW / 2];
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
+        for (int c4 = 0; c4 < CW / 4; ++c4) {
           const float4 ls = lse4[c4], dl = del4[c4];
           const float lsv[4] = {ls.x, ls.y, ls.z, ls.w}, dlv[4] = {dl.x, dl.y, dl.z, dl.w};
           float pf[4], df[4];
@@ -282,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
             const float x = fmaf(__uint_as_float(sv[cl]), sl2, -lsv[e]);
             float p = (!kMask && use_poly && poly_col<COWA_DKDV_POLY_MASK>(cl)) ? exp2_fma(x) : ptx::ex2(x);
             if (kMask) {
-              const int t = t0 + 32 * half + cl;
+              const int t = t0 + CW * part + cl;
               if (!(t >= s && t < t_hi)) p = 0.f;
             }
             pf[e] = p;
@@ -293,9 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
           dw[2 * c4] = ptx::pack_bf16(df[0], df[1]);
           dw[2 * c4 + 1] = ptx::pack_bf16(df[2], df[3]);
         }
-        // packed columns of this warp's 32 query columns lie inside the columns it just read
-        ptx::tmem_st16(buf + kColPT + 16 * half, pw);
-        ptx::tmem_st16(buf + kColDST + 16 * half, dw);
+        // packed columns of this warp's query columns: the upper half of the columns it just read
+        if constexpr (CW == 32) {
+          ptx::tmem_st16(buf + CW * part + CW / 2, pw);
+          ptx::tmem_st16(buf + 64 + CW * part + CW / 2, dw);
+        } else {
+          ptx::tmem_st8(buf + CW * part + CW / 2, pw);
+          ptx::tmem_st8(buf + 64 + CW * part + CW / 2, dw);
+        }
       };
       if (need_mask) body(std::true_type{});
       else body(std::false_type{});
@@ -306,19 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
     }
     if (ok && nsteps > 0 && ptx::mbar_wait_warp(&acc_full, 0, &abort_flag, a.status)) {
       ptx::tc_fence_after();
-      constexpr int HC = D / 2;  // accumulator columns per half
+      constexpr int HC = D / NP;  // accumulator columns of this warp
+      static_assert(HC % 32 == 0, "dV / dK columns per softmax warp must be whole 32-column loads");
       uint32_t dvv[HC], dkv[HC];
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) {
-        ptx::tmem_ld32(lane_base + Geo::kColAcc + half * HC + c * 32, dvv + c * 32);
-        ptx::tmem_ld32(lane_base + Geo::kColAcc + D + half * HC + c * 32, dkv + c * 32);
+        ptx::tmem_ld32(lane_base + Geo::kColAcc + part * HC + c * 32, dvv + c * 32);
+        ptx::tmem_ld32(lane_base + Geo::kColAcc + D + part * HC + c * 32, dkv + c * 32);
       }
       ptx::tmem_wait_ld();
       if (s < a.N) {
         __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + (int64_t)s * a.dv_st +
-                             g * a.dv_sh + half * HC;
+                             g * a.dv_sh + part * HC;
         __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + (int64_t)s * a.dk_st +
-                             g * a.dk_sh + half * HC;
+                             g * a.dk_sh + part * HC;
 #pragma unroll
         for (int c8 = 0; c8 < HC / 8; ++c8) {
           uint32_t w[4], x[4];
@@ -337,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkdv_kernel(const __grid_cons
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kKMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, 512);
   }
@@ -600,6 +618,13 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
 #endif
 template <int D>
 constexpr int kDqParts = D == 128 ? COWA_DQ_PARTS : 2;
+// softmax warps per lane quadrant of the dK/dV kernel (64 / NP query columns each); 4 measured
+// 5% slower than 2 on B200 for this kernel
+#ifndef COWA_DKDV_PARTS
+#define COWA_DKDV_PARTS 2
+#endif
+template <int D>
+constexpr int kDkdvParts = D == 128 ? COWA_DKDV_PARTS : 2;
 
 template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
@@ -611,12 +636,13 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (stages & COWA_BWD_DKDV) {
-    auto kdkdv = bwd_dkdv_kernel<D>;
+    constexpr int NPK = kDkdvParts<D>;
+    auto kdkdv = bwd_dkdv_kernel<D, NPK>;
     if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemKV)) != cudaSuccess)
       return e;
     const long long n_kv = (long long)nq * a.Hkv * a.B;
     if (n_kv > 0x7fffffffLL) return cudaErrorInvalidValue;
-    kdkdv<<<(unsigned)n_kv, kThreads, Geo::kSmemKV, s>>>(a);
+    kdkdv<<<(unsigned)n_kv, (4 * NPK + 2) * 32, Geo::kSmemKV, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (stages & COWA_BWD_DQ) {
