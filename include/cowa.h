@@ -112,6 +112,20 @@ cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int
                            int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, float* lse,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* ---- packed variable-length batch (forward) -------------------------------------------------
+ * n_seq sequences packed along the token axis: sequence s is rows cu_seqlens[s] ..
+ * cu_seqlens[s+1]-1 of q [total, H_q, d], k and v [total, H_kv, d] (cowa_tensor strides; stride_b
+ * unused but validated), at positions 0 .. len_s-1 each; o [total, H_q, d]; lse fp32
+ * contiguous [H_q, total].  Each sequence gets exactly cowa_fwd over its own rows.
+ * cu_seqlens: device int32 [n_seq + 1], non-decreasing from 0 to total (entries outside
+ * [0, total] are clamped on the device, so a malformed array cannot make the kernel touch rows
+ * outside the tensors).  Workspace: cowa_fwd_varlen_workspace_size (status word + per-sequence
+ * tile offsets, computed on the device in the same stream).  Errors as for cowa_fwd. */
+size_t cowa_fwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d);
+cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d,
+                            const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+                            float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- backward ---------------------------------------------------------------------------
  * Gradients of sum(dO * O) for the forward above, from the saved o and lse.
  * Inputs  q, k, v, o, lse as produced/consumed by cowa_fwd; dO [B, N, H_q, d] bf16.

@@ -6,8 +6,9 @@ caller-owned outputs and workspace with torch, and raises on any non-OK
 status.  There is no fallback: if libcowa.so is missing or fails to load,
 every call raises.
 
-Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_bwd,
-cowa_decode, plus the planner introspection helpers.
+Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_fwd_chunk,
+cowa_fwd_varlen, cowa_bwd, cowa_decode, cowa_decode_compact (with compact_cache /
+compact_append), cowa_decode_noalloc, plus the planner introspection helpers.
 """
 
 from __future__ import annotations
@@ -24,10 +25,6 @@ LIB_PATH = os.path.join(_HERE, "libcowa.so")
 COWA_OK = 0
 _STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED", 3: "COWA_ERR_ALIGNMENT",
            4: "COWA_ERR_WORKSPACE", 5: "COWA_ERR_CUDA", 6: "COWA_ERR_TIMEOUT"}
-
-EXPORTED = ["cowa_fwd_workspace_size", "cowa_fwd", "cowa_bwd_workspace_size", "cowa_bwd",
-            "cowa_decode_workspace_size", "cowa_decode", "cowa_workspace_status", "cowa_status_string",
-            "cowa_visible_counts", "cowa_plan_debug", "cowa_version", "cowa_decode_noalloc", "cowa_bwd_stages", "cowa_debug_wait_timeout"]
 
 BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 1, 2, 4
 
@@ -84,6 +81,10 @@ def lib() -> ctypes.CDLL:
     L.cowa_fwd.restype = i
     L.cowa_fwd_chunk.argtypes = [P, i, i, i, i, i, i, i, T, T, T, T, vp, vp, sz, vp]
     L.cowa_fwd_chunk.restype = i
+    L.cowa_fwd_varlen_workspace_size.argtypes = [P, i, i, i, i, i]
+    L.cowa_fwd_varlen_workspace_size.restype = sz
+    L.cowa_fwd_varlen.argtypes = [P, i, i, i, i, i, vp, T, T, T, T, vp, vp, sz, vp]
+    L.cowa_fwd_varlen.restype = i
     L.cowa_bwd_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_bwd_workspace_size.restype = sz
     L.cowa_bwd.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
@@ -210,6 +211,35 @@ def cowa_fwd_chunk(q, k, v, pattern: Pattern, q_offset: int, n_k=None, kv_layout
     _check("cowa_fwd_chunk", L.cowa_fwd_chunk(ctypes.byref(pat), B, Nq, int(n_k), int(q_offset), Hq, Hkv, d, _t4(q),
                                               _t4(kt), _t4(vt), _t4(out), lse.data_ptr(), workspace.data_ptr(),
                                               workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def cowa_fwd_varlen(q, k, v, cu_seqlens, pattern: Pattern, out=None, lse=None, workspace=None, stream=None):
+    """Packed variable-length batch: q [total, H_q, d], k, v [total, H_kv, d], cu_seqlens CUDA int32
+    [n_seq + 1]; returns o [total, H_q, d] bf16 and lse [H_q, total] fp32, each sequence attending
+    over its own rows at positions 0.. ."""
+    import torch
+
+    for n_, x_ in (("q", q), ("k", k), ("v", v)):
+        _bf16_cuda(n_, x_)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D CUDA int32 tensor")
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    n_seq = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device)
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_fwd_varlen_workspace_size(ctypes.byref(pat), n_seq, total, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q.device)
+    t4 = lambda x: _t4(x.unsqueeze(0))
+    _check("cowa_fwd_varlen", L.cowa_fwd_varlen(ctypes.byref(pat), n_seq, total, Hq, Hkv, d, cu_seqlens.data_ptr(),
+                                                t4(q), t4(k), t4(v), t4(out), lse.data_ptr(), workspace.data_ptr(),
+                                                workspace.numel(), _stream(stream)))
     return out, lse
 
 

@@ -298,6 +298,43 @@ cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int
   return launch_fwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
 }
 
+size_t cowa_fwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d) {
+  Pat p;
+  if (n_seq < 1 || check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, total, Hq, Hkv, d) != COWA_OK) return 0;
+  return kWsHeader + fwd_varlen_workspace_bytes(n_seq);
+}
+
+cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d,
+                            const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+                            float* lse, void* ws, size_t ws_bytes, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(1, total, Hq, Hkv, d));
+  if (n_seq < 1 || !cu_seqlens || !lse) return COWA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return COWA_ERR_ALIGNMENT;
+  COWA_TRY(check_tensor(q));
+  COWA_TRY(check_tensor(k));
+  COWA_TRY(check_tensor(v));
+  COWA_TRY(check_tensor(o));
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_fwd_varlen_workspace_size(pat, n_seq, total, Hq, Hkv, d)));
+
+  FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.pat = p; a.B = 1; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.Nq = total; a.Nk = total; a.q_off = 0;
+  a.varlen = 1; a.n_seq = n_seq; a.total = total; a.cu_seqlens = cu_seqlens;
+  a.tile_off = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.o = o.ptr; a.o_sb = 0; a.o_st = o.stride_t; a.o_sh = o.stride_h;
+  a.lse = lse;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f;
+  if (!make_tmap_bf16(&a.tm_q, q.ptr, d, total, Hq, 1, q.stride_t, q.stride_h, q.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_k, k.ptr, d, total, Hkv, 1, k.stride_t, k.stride_h, k.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_v, v.ptr, d, total, Hkv, 1, v.stride_t, v.stride_h, v.stride_b, 128))
+    return COWA_ERR_CUDA;
+  return launch_fwd(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------------------ backward
 size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d) {
   Pat p;

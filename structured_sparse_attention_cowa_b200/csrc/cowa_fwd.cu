@@ -84,9 +84,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   // ---- work item: heaviest (last) query tiles first; all heads/pairs of one tile adjacent
   const int grp = a.Hq / a.Hkv;
   const int npair = (grp + 1) >> 1;
-  const int nq = (a.Nq + kBM - 1) / kBM;
   const int per_i = a.B * a.Hkv * npair;
-  const int i = nq - 1 - (int)(blockIdx.x / per_i);
+  int i, row0 = 0, Nq = a.Nq, Nk = a.Nk, q_off = a.q_off;  // row0: first row of the sequence
+  if (!a.varlen) {
+    i = (a.Nq + kBM - 1) / kBM - 1 - (int)(blockIdx.x / per_i);
+  } else {
+    // the grid is an upper bound on the q-tiles of the packed batch: find this CTA's sequence
+    const int tiles = a.tile_off[a.n_seq];
+    const int tg = tiles - 1 - (int)(blockIdx.x / per_i);
+    if (tg < 0) return;  // whole CTA, before any barrier or TMEM use
+    int lo = 0, hi = a.n_seq - 1;  // largest s with tile_off[s] <= tg
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.tile_off[mid] <= tg) lo = mid; else hi = mid - 1;
+    }
+    i = tg - a.tile_off[lo];
+    const int st = imin(imax(a.cu_seqlens[lo], 0), a.total);
+    const int en = imin(imax(a.cu_seqlens[lo + 1], st), a.total);
+    row0 = st;
+    Nq = Nk = en - st;
+    q_off = 0;
+  }
   int rem = blockIdx.x % per_i;
   const int pair = rem % npair; rem /= npair;
   const int g = rem % a.Hkv;
@@ -94,7 +112,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   const int h0 = g * grp + 2 * pair;
   const bool has1 = (2 * pair + 1) < grp;
   // query rows of the tile: local q rows [i*BM, ...), absolute positions [t0, t1)
-  const int t0 = a.q_off + i * kBM, t1 = imin(a.q_off + a.Nq, t0 + kBM);
+  const int t0 = q_off + i * kBM, t1 = imin(q_off + Nq, t0 + kBM);
   const Range iv = interval_of(a.pat, g);
   const Tiles T = plan_tiles(a.pat, iv, t0, t1);
 
@@ -134,8 +152,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       ptx::tma_prefetch_desc(&a.tm_v);
       ptx::mbar_arrive_expect_tx(&q_full, (has1 ? 2 : 1) * Geo::kQBytes);
       for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, i * kBM, h0, b);
-        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, i * kBM, h0 + 1, b);
+        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0, b);
+        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0 + 1, b);
       }
       TileCursor cur;
       cur.init(T);
@@ -147,7 +165,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         uint8_t* dst = sRing + s * Geo::kKVBytes;
         ptx::mbar_arrive_expect_tx(&kv_full[s], Geo::kKVBytes);
         for (int u = 0; u < D / 64; ++u)
-          ptx::tma_load_4d(dst + u * 16384, is_v ? &a.tm_v : &a.tm_k, &kv_full[s], u * 64, cur.j * kBN, g, b);
+          ptx::tma_load_4d(dst + u * 16384, is_v ? &a.tm_v : &a.tm_k, &kv_full[s], u * 64, row0 + cur.j * kBN, g, b);
         if (is_v) cur.next(T);
         issued = idx + 1;
       }
@@ -251,7 +269,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       cur.init(T);
       for (int n = 0; n < ntiles; ++n, cur.next(T)) {
         const int s0 = cur.j * kBN;
-        const bool need_mask = (s0 + kBN > a.Nk) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.Nk, s0 + kBN));
+        const bool need_mask = (s0 + kBN > Nk) || !tile_full(a.pat, iv, t0, t1, s0, imin(Nk, s0 + kBN));
         if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
         // visible key columns of row t within [s0, s0+128), relative to s0 (partial tiles only)
@@ -346,10 +364,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], 0, &abort_flag, a.status)) {
         ptx::tc_fence_after();
         const float inv = 1.f / l;
-        const int rl = t - a.q_off;  // local query row
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)rl * a.o_st +
-                              (size_t)(h0 + k) * a.o_sh;
-        if (t < t1) a.lse[((size_t)b * a.Hq + h0 + k) * a.Nq + rl] = (m_used + log2f(l)) * 0.69314718055994530942f;
+        const int rl = t - q_off;  // query row within the call's (or the sequence's) rows
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb +
+                              (size_t)(row0 + rl) * a.o_st + (size_t)(h0 + k) * a.o_sh;
+        // lse: [B, H_q, N_q], or [H_q, total] for a packed batch
+        const size_t lse_i = a.varlen ? (size_t)(h0 + k) * a.total + row0 + rl
+                                      : ((size_t)b * a.Hq + h0 + k) * a.Nq + rl;
+        if (t < t1) a.lse[lse_i] = (m_used + log2f(l)) * 0.69314718055994530942f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t ov[32];
@@ -379,6 +400,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   }
 }
 
+// tile_off[s] = q-tiles of the sequences before s (lengths clamped into [0, total]); one thread:
+// the scan is over the handful of sequences of one batch
+__global__ void varlen_tiles_kernel(const int32_t* cu, int n_seq, int total, int32_t* tile_off) {
+  if (threadIdx.x != 0) return;
+  int off = 0;
+  for (int s = 0; s < n_seq; ++s) {
+    tile_off[s] = off;
+    const int st = imin(imax(cu[s], 0), total);
+    const int en = imin(imax(cu[s + 1], st), total);
+    off += (en - st + kBM - 1) / kBM;
+  }
+  tile_off[n_seq] = off;
+}
+
 template <int D>
 cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   using Geo = FwdGeom<D>;
@@ -386,8 +421,10 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
   if (e != cudaSuccess) return e;
   const int grp = a.Hq / a.Hkv;
-  const int nq = (a.Nq + kBM - 1) / kBM;
-  const long long nblk = (long long)nq * a.B * a.Hkv * ((grp + 1) / 2);
+  // packed batch: an upper bound on the q-tiles (sum of ceil(len/BM) <= total/BM + n_seq); the
+  // tile offsets are computed on the device first
+  const long long nq = a.varlen ? (long long)a.total / kBM + a.n_seq : (a.Nq + kBM - 1) / kBM;
+  const long long nblk = nq * a.B * a.Hkv * ((grp + 1) / 2);
   if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
   // the in-kernel register split assumes the compiled count equals the launch allocation
   static int regs_ok = -1;
@@ -397,11 +434,17 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
     regs_ok = fa.numRegs == kRegsLaunch ? 1 : 0;
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
+  if (a.varlen) {
+    varlen_tiles_kernel<<<1, 32, 0, s>>>(a.cu_seqlens, a.n_seq, a.total, a.tile_off);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   kern<<<(unsigned)nblk, kFwdThreads, Geo::kSmem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+size_t fwd_varlen_workspace_bytes(int n_seq) { return ((size_t)(n_seq + 1) * sizeof(int32_t) + 255) / 256 * 256; }
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s) {
   if (a.d == 64) return launch_fwd_d<64>(a, s);

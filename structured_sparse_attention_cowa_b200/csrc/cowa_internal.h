@@ -65,6 +65,11 @@ struct FwdArgs {
   Pat pat;
   int B, Hq, Hkv, d;
   int Nq, Nk, q_off;  // query rows q_off .. q_off+Nq-1 (absolute positions) against keys 0 .. Nk-1
+  // packed variable-length batch (varlen != 0): sequence s holds rows cu_seqlens[s] ..
+  // cu_seqlens[s+1]-1 of q, k, v, o (B = 1) at positions 0..; tile_off[s] = q-tiles before it
+  int varlen, n_seq, total;
+  const int32_t* cu_seqlens;
+  int32_t* tile_off;
   void* o;
   int64_t o_sb, o_st, o_sh;
   float* lse;
@@ -73,6 +78,7 @@ struct FwdArgs {
   CUtensorMap tm_q, tm_k, tm_v;
 };
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s);
+size_t fwd_varlen_workspace_bytes(int n_seq);
 
 // ---- backward ----
 struct BwdArgs {

@@ -180,6 +180,19 @@ def test_compact_entry_points_reject_bad_arguments():
                                  0x70000, n - 1, None) == 4
 
 
+def test_fwd_varlen_rejects_bad_arguments_before_launch():
+    L = cw.lib()
+    p = cw.Pattern(64, 8, 1024, 4).c()
+    n = L.cowa_fwd_varlen_workspace_size(ctypes.byref(p), 3, 1000, 8, 4, 128)
+    assert n >= 256 + 16
+    args = (ctypes.byref(p), 3, 1000, 8, 4, 128)
+    assert L.cowa_fwd_varlen(*args, None, _t(), _t(), _t(), _t(), 0x20000, 0x40000, n, None) == 1      # no cu_seqlens
+    assert L.cowa_fwd_varlen(*args, 0x30002, _t(), _t(), _t(), _t(), 0x20000, 0x40000, n, None) == 3   # misaligned
+    assert L.cowa_fwd_varlen(*args, 0x30000, _t(), _t(), _t(), _t(), 0x20000, 0x40000, n - 1, None) == 4  # workspace
+    assert L.cowa_fwd_varlen(ctypes.byref(p), 0, 1000, 8, 4, 128, 0x30000, _t(), _t(), _t(), _t(), 0x20000, 0x40000,
+                             n, None) == 1                                                          # no sequences
+
+
 def test_decode_and_bwd_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(64, 8, 1024, 4).c()

@@ -271,3 +271,25 @@ def test_device_wait_timeout_is_reported_and_context_survives(cuda_device):
     assert cw.workspace_status(ws) == 6          # COWA_ERR_TIMEOUT, and the word is cleared
     assert cw.workspace_status(ws) == 0
     _check_fwd_full(1, 300, 4, 2, 64, cw.Pattern(8, 32, 300, 2), cuda_device, extra=5)
+
+
+def test_fwd_varlen_packed_batch(cuda_device):
+    """Five sequences (1, 127, 128, 300 and 1000 tokens, plus an empty one) packed along the token
+    axis: each sequence's rows equal the oracle's forward over that sequence alone."""
+    Hq, Hkv, d = 10, 2, 128
+    pat = cw.Pattern(32, 200, 1000, 2)
+    lens = [1, 127, 0, 128, 300, 1000]
+    total = sum(lens)
+    q64, q = host_and_device((1, total, Hq, d), "q", cuda_device, 29)
+    k64, k = host_and_device((1, total, Hkv, d), "k", cuda_device, 29)
+    v64, v = host_and_device((1, total, Hkv, d), "v", cuda_device, 29)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    o, lse = cw.cowa_fwd_varlen(q[0], k[0], v[0], torch.tensor(cu, device=cuda_device), pat)
+    torch.cuda.synchronize()
+    for s_, (a_, b_) in enumerate(zip(cu[:-1], cu[1:])):
+        if b_ == a_:
+            continue
+        want_o, want_l = orc.attention_fwd(q64[:, a_:b_], k64[:, a_:b_], v64[:, a_:b_], oracle_pattern(pat))
+        err_o = np.abs(to64(o[a_:b_]) - want_o[0]).max()
+        err_l = np.abs(lse[:, a_:b_].cpu().numpy().astype(np.float64) - want_l[0]).max()
+        assert err_o <= O_ATOL and err_l <= LSE_ATOL, (s_, err_o, err_l)
