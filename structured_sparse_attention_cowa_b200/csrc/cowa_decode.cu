@@ -18,6 +18,12 @@
 //     partial per (b, h, split).
 // A second kernel merges the splits of each (b, h) (max / rescaled sums, warp shuffles)
 // and writes bf16 o and the fp32 lse.
+//
+// The same kernel reads a compacted per-head cache (sink, band ring, own interval; see
+// CompactGeom): the visible positions then form three disjoint sets, each read from its own
+// region in 64-aligned blocks (64 consecutive rows), with positions outside the CTA's chunk
+// masked.  Two small kernels keep that cache: one builds it from a prefill's K/V, one appends
+// a decoded token to every region that holds its position.
 #include <cuda_bf16.h>
 #include <math.h>
 

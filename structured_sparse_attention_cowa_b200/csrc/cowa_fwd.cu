@@ -7,9 +7,13 @@
 // the mask depends on g only.  Warp roles (12 warps = 3 warpgroups):
 //   warps 0-3  softmax for head slot 0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax for head slot 1
-//   warp  8    TMA producer: Q once, then K_j, V_j of every visited KV tile into a 4-deep ring
-//   warp  9    tcgen05 MMA issuer (one lane): S = Q K^T into TMEM, O += P V into TMEM
+//   warp  8    TMA producer: Q once, then K_j, V_j of every visited KV tile into a 5-slot ring
+//   warp  9    tcgen05 MMA issuer (the whole warp walks the loop, one elected lane issues):
+//              S = Q K^T into TMEM, O += P V into TMEM
 //   warps 10-11 idle (they complete the third warpgroup)
+// The same kernel serves a block of queries at an offset against keys already written
+// (chunked prefill: query rows q_off.., keys 0..Nk-1) and packed variable-length batches (each
+// CTA finds its sequence in per-sequence tile offsets and works on that sequence's rows).
 // Registers: the kernel is compiled for 168 per thread (384 * 168 = 64512 at launch); the two
 // softmax warpgroups then raise theirs to 216 and the third lowers to 72
 // (2*128*216 + 128*72 = 64512), so a whole 128-column score row stays in registers.  The
