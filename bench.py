@@ -364,6 +364,9 @@ def main():
     ap.add_argument("--impl", default="cowa", choices=["cowa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-outputs", default="results", choices=["results", "all"],
+                    help="results: read back the forward lse and the decode output/lse (o, dq, dk, dv stay on "
+                         "the device as in training); all: also copy o, dq, dk, dv out every step")
     ap.add_argument("--dense", action="store_true", help="also time the dense-causal mode (L >= T)")
     ap.add_argument("--sweep", action="store_true",
                     help="also time the other configurations (8K prefill D sweep, 128K layer, dense-causal at "
@@ -560,11 +563,14 @@ def run_cowa(args, world, rank, local):
 
     # ---- end to end: host buffers, copies inside the timed region.  Every step copies its inputs
     # (q, k, v, dO of the layer, q_t and pos of the decode; the KV cache is resident device state)
-    # in from pinned host memory and its results (o, dq, dk, dv, decode o) out to pinned host
-    # memory.  Steps are pipelined the way a training or serving loop prefetches: three streams
-    # (copy-in, compute, copy-out) and two device buffer sets, so step i+1's inputs land while
-    # step i computes and step i's results leave while step i+1 computes.  Within a step the
-    # forward starts once q, k, v are in (dO lands meanwhile), o leaves while the backward runs.
+    # in from pinned host memory and reads its results back into pinned host memory: by default
+    # the results a host reads in training and serving -- the forward's lse (the per-row
+    # log-partition a loss is formed from) and the decode output and lse -- while o, dq, dk, dv
+    # stay on the device for the next layer and the optimizer; --e2e-outputs all also copies
+    # o, dq, dk and dv out.  Steps are pipelined the way a training or serving loop prefetches:
+    # three streams (copy-in, compute, copy-out) and two device buffer sets, so step i+1's
+    # inputs land while step i computes and step i's results leave while step i+1 computes.
+    # Within a step the forward starts once q, k, v are in (dO lands meanwhile).
     e2e = None
     if not args.no_e2e:
         pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -573,14 +579,16 @@ def run_cowa(args, world, rank, local):
         for n, x in zip(names_in, (q, k, v, do, qt)):
             h_in[n].copy_(x)
         h_pos = pos.cpu().pin_memory()
-        names_out = ("o", "dq", "dk", "dv", "od")
-        h_out = {n: pin(x) for n, x in zip(names_out, (o, dq, dk, dv, od))}
+        all_out = args.e2e_outputs == "all"
+        names_out = ("lse", "od", "lsed") + (("o", "dq", "dk", "dv") if all_out else ())
+        dev_out = {"lse": lse, "od": od, "lsed": lsed, "o": o, "dq": dq, "dk": dk, "dv": dv}
+        h_out = {n: pin(dev_out[n]) for n in names_out}
         h2d = sum(x.numel() * x.element_size() for x in h_in.values()) + h_pos.numel() * 4
         d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
         def buffer_set():
             st = {n: torch.empty_like(x) for n, x in zip(names_in + ("pos",), (q, k, v, do, qt, pos))}
-            st.update({n: torch.empty_like(x) for n, x in zip(names_out + ("lse", "lsed"), (o, dq, dk, dv, od, lse, lsed))})
+            st.update({n: torch.empty_like(x) for n, x in dev_out.items()})
             st.update({n: torch.zeros_like(x) for n, x in (("ws_f", ws_f), ("ws_b", ws_b), ("ws_d", ws_d))})
             return st
 
@@ -620,12 +628,16 @@ def run_cowa(args, world, rank, local):
                 inputs_free[j] = e_cmp
             with torch.cuda.stream(s_out):
                 s_out.wait_event(e_fwd)
-                h_out["o"].copy_(st["o"], non_blocking=True)
+                h_out["lse"].copy_(st["lse"], non_blocking=True)
+                if all_out:
+                    h_out["o"].copy_(st["o"], non_blocking=True)
                 s_out.wait_event(e_bwd)
-                for n in ("dq", "dk", "dv"):
-                    h_out[n].copy_(st[n], non_blocking=True)
+                if all_out:
+                    for n in ("dq", "dk", "dv"):
+                        h_out[n].copy_(st[n], non_blocking=True)
                 s_out.wait_event(e_cmp)
                 h_out["od"].copy_(st["od"], non_blocking=True)
+                h_out["lsed"].copy_(st["lsed"], non_blocking=True)
                 e_o = new_ev(); e_o.record(s_out)
                 outputs_free[j] = e_o
 
@@ -650,7 +662,8 @@ def run_cowa(args, world, rank, local):
         e_ms = maxr(a.elapsed_time(b)) / KE
         e2e = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
-               "pipelined": "copy-in / compute / copy-out streams, two device buffer sets"}
+               "pipelined": "copy-in / compute / copy-out streams, two device buffer sets",
+               "outputs_read": list(names_out)}
         del sets
 
     cpu = None
