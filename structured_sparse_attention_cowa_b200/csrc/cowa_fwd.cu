@@ -80,6 +80,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   __shared__ __align__(8) uint64_t kv_full[kRingMax], kv_empty[kRingMax];
   __shared__ __align__(8) uint64_t s_full[2], p_ready[2], o_done[2];
   __shared__ __align__(8) uint64_t mma_final;
+  // single-head tile (odd GQA group): softmax 1's running max and sum per row for the merge
+  __shared__ __align__(8) uint64_t merge_ready;
+  __shared__ float merge_m[kBM], merge_l[kBM];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       ptx::mbar_init(&o_done[k], 1);
     }
     ptx::mbar_init(&mma_final, 1);
+    ptx::mbar_init(&merge_ready, 4);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -189,8 +193,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
     const uint64_t v_desc = ptx::smem_desc_sw128(ptx::smem_u32(sRing), 16384, 1024);
     const int nslot = has1 ? 2 : 1;
 
-    auto issue_s = [&](int k, int kslot) {
-      const uint64_t qd = ptx::desc_advance(q_desc, k * Geo::kQBytes);
+    auto issue_s = [&](int k, int kslot, int qk) {  // S_k = Q_qk K^T
+      const uint64_t qd = ptx::desc_advance(q_desc, qk * Geo::kQBytes);
       const uint64_t kd = ptx::desc_advance(k_desc, kslot * Geo::kKVBytes);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -210,13 +214,70 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
 
     bool ok = ptx::mbar_wait_warp(&q_full, 0, &abort_flag, a.status);
     ptx::tc_fence_after();
-    for (int n = 0; ok && n < ntiles; ++n) {
+    if (nslot == 1) {
+      // One query head (odd group): the two softmax warpgroups take alternate KV tiles of it,
+      // slot 0 the even ones and slot 1 the odd ones, each with its own running max, sum and
+      // O accumulator (merged at the end), so the tensor core still alternates between two
+      // softmaxes.  Iteration j: S0(2j), PV1(2j-1), S1(2j+1), PV0(2j).
+      const int n0cnt = (ntiles + 1) / 2, n1cnt = ntiles / 2;
+      for (int j = 0; ok && j < n0cnt; ++j) {
+        const int ne = 2 * j, no = 2 * j + 1;
+        const int kidx0 = 2 * ne, vidx0 = kidx0 + 1, kidx1 = 2 * no;
+        if (!(ok = ptx::mbar_wait_warp(&kv_full[kidx0 % Geo::kRing], (kidx0 / Geo::kRing) & 1, &abort_flag,
+                                       a.status)))
+          break;
+        ptx::tc_fence_after();
+        issue_s(0, kidx0 % Geo::kRing, 0);
+        ptx::mma_commit_warp(&s_full[0]);
+        ptx::mma_commit_warp(&kv_empty[kidx0 % Geo::kRing]);
+        if (j > 0) {  // PV1 of the previous odd tile 2j-1 (odd-tile index j-1)
+          const int pv = 2 * (2 * j - 1) + 1;
+          if (!(ok = ptx::mbar_wait_warp(&kv_full[pv % Geo::kRing], (pv / Geo::kRing) & 1, &abort_flag, a.status)))
+            break;
+          if (!(ok = ptx::mbar_wait_warp(&p_ready[1], (j - 1) & 1, &abort_flag, a.status))) break;
+          ptx::tc_fence_after();
+          issue_pv(1, pv % Geo::kRing, j - 1 > 0);
+          ptx::mma_commit_warp(&kv_empty[pv % Geo::kRing]);
+        }
+        if (no < ntiles) {
+          if (!(ok = ptx::mbar_wait_warp(&kv_full[kidx1 % Geo::kRing], (kidx1 / Geo::kRing) & 1, &abort_flag,
+                                         a.status)))
+            break;
+          ptx::tc_fence_after();
+          issue_s(1, kidx1 % Geo::kRing, 0);
+          ptx::mma_commit_warp(&s_full[1]);
+          ptx::mma_commit_warp(&kv_empty[kidx1 % Geo::kRing]);
+        }
+        if (!(ok = ptx::mbar_wait_warp(&kv_full[vidx0 % Geo::kRing], (vidx0 / Geo::kRing) & 1, &abort_flag,
+                                       a.status)))
+          break;
+        if (!(ok = ptx::mbar_wait_warp(&p_ready[0], j & 1, &abort_flag, a.status))) break;
+        ptx::tc_fence_after();
+        issue_pv(0, vidx0 % Geo::kRing, j > 0);
+        ptx::mma_commit_warp(&kv_empty[vidx0 % Geo::kRing]);
+      }
+      if (ok && ntiles > 0) {
+        ptx::mma_commit_warp(&o_done[0]);
+        if (ntiles % 2 == 0) {  // the last odd tile's PV1 is still to issue
+          const int no = ntiles - 1, pv = 2 * no + 1;
+          ok = ptx::mbar_wait_warp(&kv_full[pv % Geo::kRing], (pv / Geo::kRing) & 1, &abort_flag, a.status) &&
+               ptx::mbar_wait_warp(&p_ready[1], (n1cnt - 1) & 1, &abort_flag, a.status);
+          if (ok) {
+            ptx::tc_fence_after();
+            issue_pv(1, pv % Geo::kRing, n1cnt - 1 > 0);
+            ptx::mma_commit_warp(&kv_empty[pv % Geo::kRing]);
+          }
+        }
+        if (ok && n1cnt > 0) ptx::mma_commit_warp(&o_done[1]);
+      }
+    }
+    for (int n = 0; ok && nslot == 2 && n < ntiles; ++n) {
       const int kidx = 2 * n, vidx = 2 * n + 1;
       const int kslot = kidx % Geo::kRing, vslot = vidx % Geo::kRing;
       if (!(ok = ptx::mbar_wait_warp(&kv_full[kslot], (kidx / Geo::kRing) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
       // S0(n): P0(n-1) was consumed by PV0(n-1), issued earlier
-      issue_s(0, kslot);
+      issue_s(0, kslot, 0);
       ptx::mma_commit_warp(&s_full[0]);
       if (nslot == 2) {
         // PV1(n-1): overlaps with softmax 0 working on S0(n)
@@ -227,7 +288,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
           issue_pv(1, pv % Geo::kRing, n - 1 > 0);
           ptx::mma_commit_warp(&kv_empty[pv % Geo::kRing]);
         }
-        issue_s(1, kslot);
+        issue_s(1, kslot, 1);
         ptx::mma_commit_warp(&s_full[1]);
       }
       ptx::mma_commit_warp(&kv_empty[kslot]);
@@ -236,11 +297,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       if (!(ok = ptx::mbar_wait_warp(&p_ready[0], n & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
       issue_pv(0, vslot, n > 0);
-      if (nslot == 1) ptx::mma_commit_warp(&kv_empty[vslot]);
     }
-    if (ok && ntiles > 0) {
+    if (ok && nslot == 2 && ntiles > 0) {
       ptx::mma_commit_warp(&o_done[0]);
-      if (nslot == 2) {
+      {
         const int n = ntiles - 1, pv = 2 * n + 1;
         if (ptx::mbar_wait_warp(&p_ready[1], n & 1, &abort_flag, a.status)) {
           ptx::tc_fence_after();
@@ -258,7 +318,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
     // ------------------------------------------------------------------ softmax warpgroups
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int k = warp >> 2;  // head slot
-    if (k == 0 || has1) {
+    const bool split = !has1;  // one head: the two slots take alternate KV tiles of it
+    {
       const int r = (warp & 3) * 32 + lane;  // query row in the tile = TMEM lane
       const int t = t0 + r;
       const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -271,10 +332,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       bool ok = true;
       TileCursor cur;
       cur.init(T);
+      int cnt = 0;  // tiles of this slot so far
       for (int n = 0; n < ntiles; ++n, cur.next(T)) {
+        if (split && (n & 1) != k) continue;
         const int s0 = cur.j * kBN;
         const bool need_mask = (s0 + kBN > Nk) || !tile_full(a.pat, iv, t0, t1, s0, imin(Nk, s0 + kBN));
-        if (!(ok = ptx::mbar_wait_warp(&s_full[k], n & 1, &abort_flag, a.status))) break;
+        if (!(ok = ptx::mbar_wait_warp(&s_full[k], cnt & 1, &abort_flag, a.status))) break;
         ptx::tc_fence_after();
         // visible key columns of row t within [s0, s0+128), relative to s0 (partial tiles only)
         const int sink_end = imin(a.pat.S, t + 1) - s0;
@@ -337,7 +400,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
             m_used = m_new;
             lsum = ptx::f2_mul(lsum, ptx::f2_pack(alpha, alpha));
           }
-          if (n > 0) {
+          if (cnt > 0) {
             // O row *= alpha, a warp-collective TMEM round trip (alpha = 1 on the other lanes);
             // PV_k(n-1) has completed (the commit of S_k(n) covers it), so O_k is stable here
 #pragma unroll
@@ -360,34 +423,83 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&p_ready[k]);
+        ++cnt;
       }
       float la, lb;
       ptx::f2_unpack(lsum, la, lb);
       const float l = la + lb;
       // ---- epilogue
-      if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], 0, &abort_flag, a.status)) {
+      const int rl = t - q_off;  // query row within the call's (or the sequence's) rows
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb + (size_t)(row0 + rl) * a.o_st +
+                            (size_t)h0 * a.o_sh;
+      // lse: [B, H_q, N_q], or [H_q, total] for a packed batch
+      const size_t lse_h0 = a.varlen ? (size_t)h0 * a.total + row0 + rl : ((size_t)b * a.Hq + h0) * a.Nq + rl;
+      const size_t lse_step = a.varlen ? (size_t)a.total : (size_t)a.Nq;  // to the next head
+      if (!split) {
+        if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[k], 0, &abort_flag, a.status)) {
+          ptx::tc_fence_after();
+          const float inv = 1.f / l;
+          if (t < t1) a.lse[lse_h0 + k * lse_step] = (m_used + log2f(l)) * 0.69314718055994530942f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(o_tm + c * 32, ov);  // warp-collective: every lane loads, valid rows store
+            ptx::tmem_wait_ld();
+            if (t < t1) {
+#pragma unroll
+              for (int c8 = 0; c8 < 4; ++c8) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  w[e] = ptx::pack_bf16(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv,
+                                        __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv);
+                reinterpret_cast<uint4*>(orow + (size_t)k * a.o_sh)[c * 4 + c8] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+      } else if (k == 1) {
+        // hand this slot's running max and sum to slot 0, which merges the two halves
+        const bool have = ok && cnt > 0 && ptx::mbar_wait_warp(&o_done[1], 0, &abort_flag, a.status);
         ptx::tc_fence_after();
-        const float inv = 1.f / l;
-        const int rl = t - q_off;  // query row within the call's (or the sequence's) rows
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (size_t)b * a.o_sb +
-                              (size_t)(row0 + rl) * a.o_st + (size_t)(h0 + k) * a.o_sh;
-        // lse: [B, H_q, N_q], or [H_q, total] for a packed batch
-        const size_t lse_i = a.varlen ? (size_t)(h0 + k) * a.total + row0 + rl
-                                      : ((size_t)b * a.Hq + h0 + k) * a.Nq + rl;
-        if (t < t1) a.lse[lse_i] = (m_used + log2f(l)) * 0.69314718055994530942f;
+        merge_m[r] = have ? m_used : -INFINITY;
+        merge_l[r] = have ? l : 0.f;
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&merge_ready);
+      } else if (ok && ntiles > 0 && ptx::mbar_wait_warp(&o_done[0], 0, &abort_flag, a.status) &&
+                 ptx::mbar_wait_warp(&merge_ready, 0, &abort_flag, a.status)) {
+        // O = (O0 2^(m0-m) + O1 2^(m1-m)) / (l0 2^(m0-m) + l1 2^(m1-m)), m = max(m0, m1)
+        ptx::tc_fence_after();
+        const float m1 = merge_m[r], l1 = merge_l[r];
+        const float m = fmaxf(m_used, m1);
+        const float f0 = m_used == -INFINITY ? 0.f : ptx::ex2(m_used - m);
+        const float f1 = m1 == -INFINITY ? 0.f : ptx::ex2(m1 - m);
+        const float lt = l * f0 + l1 * f1;
+        const float inv = 1.f / lt, g0 = f0 * inv, g1 = f1 * inv;
+        const bool two = ntiles > 1;  // slot 1 has tiles (uniform over the CTA)
+        if (t < t1) a.lse[lse_h0] = (m + log2f(lt)) * 0.69314718055994530942f;
+        const uint32_t o1_tm = lane_base + Geo::kColO + D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
+          uint32_t ov[32], ow[32];
           ptx::tmem_ld32(o_tm + c * 32, ov);  // warp-collective: every lane loads, valid rows store
+          if (two) ptx::tmem_ld32(o1_tm + c * 32, ow);
           ptx::tmem_wait_ld();
           if (t < t1) {
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
               uint32_t w[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                w[e] = ptx::pack_bf16(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv,
-                                      __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv);
+              for (int e = 0; e < 4; ++e) {
+                const int i0 = c8 * 8 + 2 * e;
+                float x0 = __uint_as_float(ov[i0]) * g0, x1 = __uint_as_float(ov[i0 + 1]) * g0;
+                if (two) {
+                  x0 += __uint_as_float(ow[i0]) * g1;
+                  x1 += __uint_as_float(ow[i0 + 1]) * g1;
+                }
+                w[e] = ptx::pack_bf16(x0, x1);
+              }
               reinterpret_cast<uint4*>(orow)[c * 4 + c8] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
