@@ -68,6 +68,36 @@ def test_visible_counts_bit_exact(N, Hkv, BM, BN, pat):
     assert np.array_equal(got, want)
 
 
+def _random_plan_cases(n, seed):
+    """Seeded random configurations across the planner's edge classes: T - S not divisible by H,
+    S = 0, S >= T (no intervals), L = 1, L >= T (dense causal), N < T and N > T, tile sizes
+    32 / 64 / 128, duplicated windows (D < H) and a KV-head offset (tensor-parallel rank)."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for _ in range(n):
+        H = int(rng.choice([1, 2, 3, 4, 6, 8]))
+        D = int(rng.choice([x for x in range(1, H + 1) if H % x == 0]))
+        N = int(rng.integers(1, 520))
+        T = int(rng.integers(1, 640))
+        S = int(rng.choice([0, int(rng.integers(0, T + 1)), T]))
+        L = int(rng.choice([1, int(rng.integers(1, 200)), T + 5]))
+        BM, BN = int(rng.choice([32, 64, 128])), int(rng.choice([32, 64, 128]))
+        P = int(rng.choice([1, 2])) if H % 2 == 0 else 1  # ranks sharing the H KV heads
+        Hkv = H // P
+        base = int(rng.integers(0, P)) * Hkv
+        pat = cw.Pattern(S, L, T, D, kv_head_base=base, h_kv_global=H if P > 1 else 0)
+        cases.append((N, Hkv, BM, BN, pat))
+    return cases
+
+
+@pytest.mark.parametrize("N,Hkv,BM,BN,pat", _random_plan_cases(40, seed=2027))
+def test_random_plans_and_counts_match_the_mask(N, Hkv, BM, BN, pat):
+    """Host forward / backward tile plans and visible counts against the oracle's explicit mask,
+    bit-exact, over random configurations."""
+    test_host_plans_match_mask_bit_exact(N, Hkv, BM, BN, pat)
+    test_visible_counts_bit_exact(N, Hkv, BM, BN, pat)
+
+
 def _closed_form_counts(N, S, L, T, H, D, g):
     """|sink U band U interval| per position by inclusion-exclusion (vectorised over t)."""
     b = [S + (i * (T - S)) // H for i in range(H + 1)]
