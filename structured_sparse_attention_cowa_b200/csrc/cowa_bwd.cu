@@ -257,10 +257,25 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
     const int t_hi = special ? a.N : imin(a.N, s + a.pat.L);  // rows [s, t_hi) see key s
     const float sl2 = a.scale_log2;
     bool ok = true;
+    // query tile of the current step and its two sub-steps' mask flags, advanced incrementally
+    // (every grp steps) instead of dividing and re-testing the tile on every sub-step
+    int i_cur = i_lo, h_cnt = 0;
+    auto masks_of = [&](int i, bool* nm) {
+      for (int x = 0; x < 2; ++x) {
+        const int u0 = i * kTile + x * kSub;
+        nm[x] = !tile_full(a.pat, iv, u0, imin(a.N, u0 + kSub), s0, s1);
+      }
+    };
+    bool nm[2];
+    masks_of(i_cur, nm);
     for (int m = 0; m < nsub; ++m) {
       const int n = m >> 1, hq = m & 1;
-      const int t0 = (i_lo + n / grp) * kTile + hq * kSub;  // first query row of the sub-step
-      const bool need_mask = !tile_full(a.pat, iv, t0, imin(a.N, t0 + kSub), s0, s1);
+      if (hq == 0 && m > 0 && ++h_cnt == grp) {
+        h_cnt = 0;
+        masks_of(++i_cur, nm);
+      }
+      const int t0 = i_cur * kTile + hq * kSub;  // first query row of the sub-step
+      const bool need_mask = nm[hq];
       if (!(ok = ptx::mbar_wait_warp(&sdp_full[m & 1], (m >> 1) & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
       const uint32_t buf = lane_base + 128 * (m & 1);
