@@ -197,6 +197,53 @@ def test_compact_cache_rows_hold_every_visible_position(pat, Hkv):
         assert rows == 20736
 
 
+@pytest.mark.parametrize("pat,Hkv", [
+    (cw.Pattern(20, 100, 2000, 2), 2),
+    (cw.Pattern(0, 70, 1800, 4), 4),
+    (cw.Pattern(64, 256, 1500, 1), 2),
+    (cw.Pattern(16, 90, 16, 2), 2),
+    (cw.Pattern(3, 9, 257, 2, kv_head_base=2, h_kv_global=4), 2),
+])
+def test_compact_layout_holds_every_visible_key_at_every_position(pat, Hkv):
+    """Replays appends position by position on the documented layout (sink row p, ring row
+    S64 + p mod R, interval row S64 + R + p - round_down64(lo)), reading the row count from the
+    library, and checks that at every decode position every key the oracle's mask makes visible
+    is still in its region, read as whole 64-aligned blocks that stay inside that region."""
+    rows = cw.lib().cowa_compact_rows(ctypes.byref(pat.c()), Hkv)
+    H = pat.h_kv_global or Hkv
+    S64 = -(-pat.S // 64) * 64
+    R = -(-pat.L // 64) * 64 + 64
+    b = orc.interval_bounds(pat.S, pat.T, H)
+    N = 700
+    op = _oracle_pattern(pat)
+    for g in range(Hkv):
+        mask_g = orc.visible_mask(np.arange(N), N, op, g, Hkv)  # [N, N]
+        G = pat.kv_head_base + g
+        slot = (G % pat.D) * (H // pat.D)
+        lo, hi = b[slot], b[slot + 1]
+        lo64 = lo // 64 * 64
+        store = {}  # row -> position held
+        for t in range(N):
+            store[S64 + t % R] = t                      # append position t
+            if t < pat.S:
+                store[t] = t
+            if lo <= t < hi:
+                store[S64 + R + t - lo64] = t
+            for s_ in np.nonzero(mask_g[t])[0]:
+                if s_ < pat.S:
+                    row, blk = s_, (s_ // 64 * 64, s_ // 64 * 64 + 64, 0, S64)
+                elif s_ > t - pat.L:
+                    row = S64 + s_ % R
+                    p0 = s_ // 64 * 64
+                    blk = (S64 + p0 % R, S64 + p0 % R + 64, S64, S64 + R)
+                else:
+                    assert lo <= s_ < hi
+                    row = S64 + R + s_ - lo64
+                    blk = (S64 + R + (s_ // 64 * 64 - lo64), S64 + R + (s_ // 64 * 64 - lo64) + 64, S64 + R, rows)
+                assert store.get(row) == s_, (g, t, s_)
+                assert blk[2] <= blk[0] and blk[1] <= blk[3], (g, t, s_, blk)
+
+
 def test_compact_entry_points_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(20, 100, 2000, 2).c()
