@@ -355,6 +355,175 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
     return out
 
 
+# ------------------------------------------------------------------------------ KV-head TP
+class TpRank:
+    """One rank's share of the layer under KV-head tensor parallelism (--shard heads).
+
+    The rank owns runs of consecutive global KV heads (`shard.kv_head_runs`); per run it holds its
+    own q, k, v, dO (the run's query heads and KV heads), outputs, decode cache and workspaces,
+    and each call passes kv_head_base = the run's first global head and h_kv_global = the layer's
+    KV-head count, so that its intervals are the ones those heads have in the whole layer."""
+
+    def __init__(self, cw, synth, torch, dev, rank: int, world: int, order: str, c=None, dc=None):
+        import ctypes
+
+        from structured_sparse_attention_cowa_b200 import shard
+
+        c, dc = c or TRAIN, dc or DECODE
+        H, grp, B, N, d = c["Hkv"], c["Hq"] // c["Hkv"], c["B"], c["N"], c["d"]
+        self.cw = cw
+        self.runs = shard.kv_head_runs(rank, world, H, grp, order)
+        lib = cw.lib()
+        self.bufs = []
+        for run in self.runs:
+            nq, nk = run.n * grp, run.n
+            ex = 100 + run.G0  # each run's heads draw their own inputs
+            pat = shard.run_pattern(cw.Pattern(c["S"], c["L"], c["T"], c["D"]), run, H)
+            dpat = shard.run_pattern(cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"]), run, H)
+            rnd = lambda shape, name: synth.cuda_normal_bf16(shape, synth.seed_of(name, ex), dev)
+            b = {"run": run, "pat": pat, "dpat": dpat,
+                 "q": rnd((B, N, nq, d), "q"), "k": rnd((B, N, nk, d), "k"), "v": rnd((B, N, nk, d), "v"),
+                 "do": rnd((B, N, nq, d), "do"),
+                 "kc": rnd((dc["B"], nk, dc["T_cap"], dc["d"]), "k_cache"),
+                 "vc": rnd((dc["B"], nk, dc["T_cap"], dc["d"]), "v_cache"),
+                 "qt": rnd((dc["B"], nq, dc["d"]), "q_t"),
+                 "pos": torch.full((dc["B"],), dc["pos"], dtype=torch.int32, device=dev)}
+            b["o"] = torch.empty_like(b["q"])
+            b["lse"] = torch.empty((B, nq, N), dtype=torch.float32, device=dev)
+            b["dq"], b["dk"], b["dv"] = torch.empty_like(b["q"]), torch.empty_like(b["k"]), torch.empty_like(b["v"])
+            b["od"] = torch.empty((dc["B"], nq, dc["d"]), dtype=torch.bfloat16, device=dev)
+            b["lsed"] = torch.empty((dc["B"], nq), dtype=torch.float32, device=dev)
+            cp, cpd = pat.c(), dpat.c()
+            ws = lambda n: torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
+            b["ws_f"] = ws(lib.cowa_fwd_workspace_size(ctypes.byref(cp), B, N, nq, nk, d))
+            b["ws_b"] = ws(lib.cowa_bwd_workspace_size(ctypes.byref(cp), B, N, nq, nk, d))
+            b["ws_d"] = ws(lib.cowa_decode_workspace_size(ctypes.byref(cpd), dc["B"], nq, nk, dc["d"], dc["T_cap"]))
+            self.bufs.append(b)
+
+    def fwd(self):
+        for b in self.bufs:
+            self.cw.cowa_fwd(b["q"], b["k"], b["v"], b["pat"], out=b["o"], lse=b["lse"], workspace=b["ws_f"])
+
+    def bwd(self):
+        for b in self.bufs:
+            self.cw.cowa_bwd(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], b["pat"], dq=b["dq"], dk=b["dk"],
+                             dv=b["dv"], workspace=b["ws_b"])
+
+    def dec(self):
+        for b in self.bufs:
+            self.cw.cowa_decode(b["qt"], b["kc"], b["vc"], b["pos"], b["dpat"], out=b["od"], lse=b["lsed"],
+                                workspace=b["ws_d"])
+
+    def statuses(self):
+        return [self.cw.workspace_status(b[w]) for b in self.bufs for w in ("ws_f", "ws_b", "ws_d")]
+
+    @property
+    def launches_per_step(self) -> int:
+        return 6 * len(self.bufs)  # per run: forward 1, backward 3, decode 2
+
+
+def run_cowa_tp(args, world, rank, local):
+    """--shard heads: the whole 32K layer and the whole 128K decode batch split by KV head over P
+    ranks (strong scaling), each rank's calls over its own runs of global KV heads.  Under
+    torchrun every process is one rank (P = WORLD_SIZE) and the step time is the max over ranks.
+    In one process, --tp-ranks P runs the P ranks' calls one rank after another on the one GPU:
+    the op has no exchange step, so each rank's device time there is the time it would take on
+    its own GPU, and `tp.projected` gives the P-GPU step as the slowest rank's time; `value` stays
+    what the one GPU did (all the work over the sum of the ranks' times)."""
+    import torch
+
+    from structured_sparse_attention_cowa_b200 import cowa as cw
+    from structured_sparse_attention_cowa_b200 import shard, synth
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    P = world if world > 1 else max(1, args.tp_ranks)
+    my_ranks = [rank] if world > 1 else list(range(P))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c, dc = TRAIN, DECODE
+    H, grp = c["Hkv"], c["Hq"] // c["Hkv"]
+    K, W = args.steps, max(3, args.warmup)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    rows, launches = [], 0
+    with ClockSampler(local) as clk:
+        for r in my_ranks:
+            tr = TpRank(cw, synth, torch, dev, r, P, args.shard_order)
+            for _ in range(W):
+                tr.fwd(); tr.bwd(); tr.dec()
+            torch.cuda.synchronize()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            torch.cuda.synchronize()
+            a.record()
+            for s in range(K):
+                e = ev[s]
+                e[0].record(); tr.fwd()
+                e[1].record(); tr.bwd()
+                e[2].record(); tr.dec()
+                e[3].record()
+            b.record()
+            torch.cuda.synchronize()
+            barrier()
+            bad = [x for x in tr.statuses() if x != 0]
+            if bad:
+                raise RuntimeError(f"device status {bad[0]} after the timed region (rank {r})")
+            avg = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in ev)
+            pairs = shard.rank_visible_pairs(cw.Pattern(c["S"], c["L"], c["T"], c["D"]), r, P, H, grp, c["N"],
+                                             c["B"], args.shard_order)
+            rows.append({"rank": r, "runs": [[x.G0, x.n] for x in tr.runs], "ms": a.elapsed_time(b) / K,
+                         "fwd_ms": avg(0, 1), "bwd_ms": avg(1, 2), "decode_ms": avg(2, 3),
+                         "visible_pairs": pairs})
+            launches += K * tr.launches_per_step
+            del tr
+            torch.cuda.empty_cache()
+
+    step_ms = max_over_ranks(max(x["ms"] for x in rows), dist, dev)
+    pairs_all = visible_pairs(c["N"], c["S"], c["L"], c["T"], c["D"], c["Hkv"], c["Hq"], c["B"])
+    flop = 14.0 * c["d"] * pairs_all  # forward 4*d + backward 10*d per visible pair, the whole layer
+    if dist is not None:
+        gathered = [None] * world
+        dist.all_gather_object(gathered, rows)
+        rows = [x for part in gathered for x in part]
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    rank_ms = [x["ms"] for x in rows]
+    rank_pairs = [x["visible_pairs"] for x in rows]
+    if world > 1:
+        value, ms_line = flop / (step_ms * 1e-3) / 1e12, step_ms
+    else:
+        ms_line = sum(rank_ms)
+        value = flop / (ms_line * 1e-3) / 1e12
+    tp = {"order": args.shard_order, "P": P, "ranks": rows,
+          "balance_pairs": statistics.mean(rank_pairs) / max(rank_pairs),
+          "balance_ms": statistics.mean(rank_ms) / max(rank_ms)}
+    if world == 1 and P > 1:
+        tp["projected"] = {"step_ms": max(rank_ms), "tflops": flop / (max(rank_ms) * 1e-3) / 1e12,
+                           "note": "each rank on its own GPU: the slowest rank's time (no exchange step)"}
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms_line, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "train 32K layer fwd+bwd + decode 128K cache, whole layer split by KV head",
+                       "train": TRAIN, "decode": DECODE, "l2": "inputs larger than L2 (126 MB); no flush",
+                       "parallelism": f"kv-head TP x{P} ({args.shard_order})" + (", ranks run in turn on one GPU"
+                                                                                 if world == 1 and P > 1 else "")},
+            "tp": tp, "roofline": None, "e2e": None, "cpu_baseline": None, "gpu_launches": launches,
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -368,6 +537,13 @@ def main():
                     help="results: read back the forward lse and the decode output/lse (o, dq, dk, dv stay on "
                          "the device as in training); all: also copy o, dq, dk, dv out every step")
     ap.add_argument("--dense", action="store_true", help="also time the dense-causal mode (L >= T)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="batch: every rank runs the per-GPU workload on its own batch element (weak scaling); "
+                         "heads: the one layer split by KV head over the ranks (strong scaling, see run_cowa_tp)")
+    ap.add_argument("--shard-order", default="folded", choices=["folded", "contiguous"],
+                    help="--shard heads: which global KV heads each rank owns (shard.head_owner)")
+    ap.add_argument("--tp-ranks", type=int, default=1,
+                    help="--shard heads in one process: run this many ranks' calls in turn on the one GPU")
     ap.add_argument("--sweep", action="store_true",
                     help="also time the other configurations (8K prefill D sweep, 128K layer, dense-causal at "
                          "32K/128K, dense decode) and add them under 'sweep' (one GPU only)")
@@ -378,6 +554,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.shard == "heads":
+        return run_cowa_tp(args, world, rank, local)
     return run_cowa(args, world, rank, local)
 
 
