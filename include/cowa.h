@@ -68,8 +68,9 @@ typedef enum {
  *   L  near-diagonal width in keys (includes the query's own key), L >= 1
  *   T  declared span: the long-range region is [S, T); T >= S
  *   D  number of distinct long-range intervals, 1 <= D, D divides h_kv_global
- *   kv_head_base  global index of this call's KV head 0 (0 on one GPU; KV-head
- *                 tensor parallelism passes r * H / P on rank r)
+ *   kv_head_base  global index of this call's KV head 0 (0 on one GPU; under KV-head
+ *                 tensor parallelism a call covers consecutive global heads G0 .. and
+ *                 passes G0: r * H / P on rank r for a contiguous split)
  *   h_kv_global   H, KV heads in the whole layer (0 means "= H_kv of the call")
  *   softmax_scale multiplier of q.k (<= 0 means 1/sqrt(d)) */
 typedef struct {
