@@ -6,6 +6,12 @@ caller-owned outputs and workspace with torch, and raises on any non-OK
 status.  There is no fallback: if libcowa.so is missing or fails to load,
 every call raises.
 
+Calls are asynchronous on the stream, as in the C ABI.  A kernel whose bounded wait
+runs out records COWA_ERR_TIMEOUT in its workspace's status word instead of hanging;
+reading that word needs a stream synchronisation, so no call reads it on its own:
+pass `workspace=` and call `workspace_status(workspace)` at a point where a sync is
+acceptable (a workspace the binding allocates itself is not checked).
+
 Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_fwd_chunk,
 cowa_fwd_varlen, cowa_bwd, cowa_decode, cowa_decode_compact (with compact_cache /
 compact_append), cowa_decode_noalloc, plus the planner introspection helpers.
