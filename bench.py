@@ -284,14 +284,20 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
 
     out = []
 
-    def timed(fn):
+    def timed(fn, inner=1):
+        """Median over `reps` of the per-call time of `inner` back-to-back calls between one pair
+        of events (inner > 1 for sub-millisecond calls, so that host launch gaps between the
+        calls overlap the device work instead of being timed)."""
         fn()
         torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(); fn(); b.record(); torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b))
+            a.record()
+            for _ in range(inner):
+                fn()
+            b.record(); torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / inner)
         return statistics.median(ts)
 
     for name, B, N, Hq, Hkv, d, S, L, T, D, do_bwd in SWEEP:
@@ -326,13 +332,32 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
         del q, k, v, o, lse
         torch.cuda.empty_cache()
 
-    # decode in the dense-causal mode: every cached token up to pos is visible
+    # decode: the CoWA pattern over the full cache, the dense-causal mode (every cached token up
+    # to pos visible) and the CoWA pattern over the compacted cache, timed alike: explicit
+    # workspaces, 10 back-to-back calls per event pair
+    import ctypes
+
     dc = DECODE
-    dpat = cw.Pattern(dc["S"], dc["T"], dc["T"], dc["D"])
+    L_ = cw.lib()
     qt = synth.cuda_normal_bf16((dc["B"], dc["Hq"], dc["d"]), synth.seed_of("q_t"), dev)
     pos = torch.full((dc["B"],), dc["pos"], dtype=torch.int32, device=dev)
     od = torch.empty((dc["B"], dc["Hq"], dc["d"]), dtype=torch.bfloat16, device=dev)
-    d_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, dpat, out=od))
+    ws_of = lambda n: torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
+    pat_c = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
+    toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
+    vbytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2
+
+    ws_c = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(pat_c.c()), dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                dc["T_cap"]))
+    f_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, pat_c, out=od, workspace=ws_c), inner=10)
+    out.append({"config": "decode 128K (full cache)", "B": dc["B"], "pos": dc["pos"], "decode_ms": f_ms,
+                "decode_gbs": vbytes / (f_ms * 1e-3) / 1e9, "decode_frac_hbm": vbytes / (f_ms * 1e-3) / 1e9 / hbm_gbs,
+                "bytes": vbytes})
+
+    dpat = cw.Pattern(dc["S"], dc["T"], dc["T"], dc["D"])
+    ws_dd = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(dpat.c()), dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
+                                                 dc["T_cap"]))
+    d_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, dpat, out=od, workspace=ws_dd), inner=10)
     dbytes = float(dc["pos"] + 1) * dc["B"] * dc["Hkv"] * dc["d"] * 2 * 2
     out.append({"config": "decode 128K dense causal", "B": dc["B"], "pos": dc["pos"], "decode_ms": d_ms,
                 "decode_gbs": dbytes / (d_ms * 1e-3) / 1e9, "decode_frac_hbm": dbytes / (d_ms * 1e-3) / 1e9 / hbm_gbs,
@@ -340,17 +365,19 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
 
     # decode over the compacted per-head cache (sink + band ring + own interval), built from the
     # full cache; the same visible bytes are read, the cache holds 20,736 instead of 131,072 rows
-    pat_c = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
     kc_c, vc_c = cw.compact_cache(kc.transpose(1, 2), vc.transpose(1, 2), pat_c)
-    c_ms = timed(lambda: cw.cowa_decode_compact(qt, kc_c, vc_c, pos, pat_c, out=od))
-    toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
-    vbytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2
+    ws_k = ws_of(L_.cowa_decode_compact_workspace_size(ctypes.byref(pat_c.c()), dc["B"], dc["Hq"], dc["Hkv"],
+                                                        dc["d"]))
+    c_ms = timed(lambda: cw.cowa_decode_compact(qt, kc_c, vc_c, pos, pat_c, out=od, workspace=ws_k), inner=10)
     rows = cw.compact_rows(pat_c, dc["Hkv"])
     out.append({"config": "decode 128K over the compacted cache", "B": dc["B"], "pos": dc["pos"], "decode_ms": c_ms,
                 "decode_gbs": vbytes / (c_ms * 1e-3) / 1e9, "decode_frac_hbm": vbytes / (c_ms * 1e-3) / 1e9 / hbm_gbs,
                 "cache_rows_per_head": rows, "full_cache_rows_per_head": dc["T_cap"],
                 "cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * rows * dc["d"] * 2,
                 "full_cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * dc["T_cap"] * dc["d"] * 2})
+    for w in (ws_c, ws_dd, ws_k):
+        if cw.workspace_status(w) != 0:
+            raise RuntimeError("device status set in the decode sweep")
     del kc_c, vc_c
     return out
 
