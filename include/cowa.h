@@ -131,7 +131,8 @@ cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H
  * Gradients of sum(dO * O) for the forward above, from the saved o and lse.
  * Inputs  q, k, v, o, lse as produced/consumed by cowa_fwd; dO [B, N, H_q, d] bf16.
  * Outputs dq [B, N, H_q, d], dk and dv [B, N, H_kv, d], bf16 (fp32 accumulation).
- * The workspace holds fp32 row statistics and fp32 gradient accumulators. */
+ * The workspace holds fp32 row statistics (Delta = rowsum(dO * O) and lse * log2(e) per
+ * query row). */
 size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d);
 cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d,
                      cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse,
@@ -151,6 +152,25 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int H_q, int 
                             cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse,
                             cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
                             int stages, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- backward of a packed variable-length batch ---------------------------------------------
+ * The gradients of cowa_fwd_varlen: n_seq sequences packed along the token axis, sequence s at
+ * rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of q, o, dO, dq [total, H_q, d] and k, v, dk, dv
+ * [total, H_kv, d] (cowa_tensor strides; stride_b unused but validated), each at positions
+ * 0 .. len_s-1; lse fp32 contiguous [H_q, total] as cowa_fwd_varlen writes it.  Each sequence gets
+ * exactly cowa_bwd over its own rows: the call runs, in stream order and one sequence after
+ * another, a strided copy of the sequence's lse rows into the workspace and the three backward
+ * kernels on row-offset views (launches grow with n_seq: 3 kernels and 1 copy per non-empty
+ * sequence).
+ * cu_seqlens: HOST int32 [n_seq + 1], cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seq] =
+ * total, every length <= max_len; otherwise COWA_ERR_INVALID_ARG (a length above max_len:
+ * COWA_ERR_WORKSPACE) before anything is enqueued.  Workspace:
+ * cowa_bwd_varlen_workspace_size(pat, max_len, ...).  Other errors as for cowa_bwd. */
+size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int max_len, int H_q, int H_kv, int d);
+cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, const int32_t* cu_seqlens, int total, int max_len,
+                            int H_q, int H_kv, int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+                            const float* lse, cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /* ---- decode (one new token per sequence, KV cache) -----------------------------------------
  * q_t    [B, H_q, d] bf16, contiguous.

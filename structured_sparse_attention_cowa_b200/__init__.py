@@ -5,9 +5,10 @@ backward kernels, a split-KV decode kernel); `cowa` is its ctypes binding.
 """
 
 from .cowa import (CowaError, Pattern, compact_append, compact_cache, compact_rows, cowa_bwd,  # noqa: F401
+                   cowa_bwd_varlen,
                    cowa_decode, cowa_decode_compact, cowa_fwd, cowa_fwd_chunk, cowa_fwd_varlen, lib, plan_debug, visible_counts,
                    workspace_status)
 
-__all__ = ["Pattern", "CowaError", "cowa_fwd", "cowa_fwd_chunk", "cowa_fwd_varlen", "cowa_bwd", "cowa_decode", "cowa_decode_compact",
+__all__ = ["Pattern", "CowaError", "cowa_fwd", "cowa_fwd_chunk", "cowa_fwd_varlen", "cowa_bwd", "cowa_bwd_varlen", "cowa_decode", "cowa_decode_compact",
            "compact_rows", "compact_cache", "compact_append", "lib", "plan_debug", "visible_counts",
            "workspace_status"]

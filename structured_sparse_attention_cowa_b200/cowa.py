@@ -13,7 +13,7 @@ pass `workspace=` and call `workspace_status(workspace)` at a point where a sync
 acceptable (a workspace the binding allocates itself is not checked).
 
 Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_fwd_chunk,
-cowa_fwd_varlen, cowa_bwd, cowa_decode, cowa_decode_compact (with compact_cache /
+cowa_fwd_varlen, cowa_bwd, cowa_bwd_varlen, cowa_decode, cowa_decode_compact (with compact_cache /
 compact_append), cowa_decode_noalloc, plus the planner introspection helpers.
 """
 
@@ -97,6 +97,10 @@ def lib() -> ctypes.CDLL:
     L.cowa_bwd.restype = i
     L.cowa_bwd_stages.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, i, vp, sz, vp]
     L.cowa_bwd_stages.restype = i
+    L.cowa_bwd_varlen_workspace_size.argtypes = [P, i, i, i, i]
+    L.cowa_bwd_varlen_workspace_size.restype = sz
+    L.cowa_bwd_varlen.argtypes = [P, i, vp, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
+    L.cowa_bwd_varlen.restype = i
     L.cowa_decode_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_decode_workspace_size.restype = sz
     L.cowa_decode.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp, sz, vp]
@@ -276,6 +280,40 @@ def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, w
                                                     _t4(o), lse.data_ptr(), _t4(do), _t4(dq), _t4(dk), _t4(dv),
                                                     stages, workspace.data_ptr(), workspace.numel(),
                                                     _stream(stream)))
+    return dq, dk, dv
+
+
+def cowa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens, pattern: Pattern, dq=None, dk=None, dv=None, workspace=None,
+                    stream=None):
+    """Gradients of cowa_fwd_varlen: q, o, do [total, H_q, d], k, v [total, H_kv, d], lse [H_q, total],
+    cu_seqlens on the HOST (list, numpy array or CPU tensor of n_seq + 1 offsets); returns dq, dk, dv.
+    One sequence after another in stream order (see cowa_bwd_varlen in cowa.h)."""
+    import torch
+
+    for n_, x_ in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _bf16_cuda(n_, x_)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                                         dtype=np.int64))
+    if cu.ndim != 1 or cu.size < 2 or cu.min() < 0 or cu.max() > 2**31 - 1:
+        raise ValueError("cu_seqlens must be a 1-D host array of n_seq + 1 offsets")
+    cu = cu.astype(np.int32)
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    n_seq = cu.size - 1
+    max_len = max(1, int(np.diff(cu).max()))
+    dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
+    dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
+    dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
+    pat = pattern.c()
+    L = lib()
+    ws_bytes = L.cowa_bwd_varlen_workspace_size(ctypes.byref(pat), max_len, Hq, Hkv, d)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, q.device)
+    t4 = lambda x: _t4(x.unsqueeze(0))
+    _check("cowa_bwd_varlen", L.cowa_bwd_varlen(ctypes.byref(pat), n_seq, cu.ctypes.data_as(ctypes.c_void_p), total,
+                                                max_len, Hq, Hkv, d, t4(q), t4(k), t4(v), t4(o), lse.data_ptr(),
+                                                t4(do), t4(dq), t4(dk), t4(dv), workspace.data_ptr(),
+                                                workspace.numel(), _stream(stream)))
     return dq, dk, dv
 
 

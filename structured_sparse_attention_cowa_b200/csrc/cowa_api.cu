@@ -386,6 +386,62 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int H
   return launch_bwd(a, stages, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------------------ packed backward
+namespace {
+// workspace of the packed backward: [header + backward statistics for max_len rows][lse scratch]
+size_t bwd_varlen_stats_bytes(int max_len, int Hq, int Hkv, int d) {
+  return kWsHeader + bwd_workspace_bytes(1, max_len, Hq, Hkv, d);
+}
+cowa_tensor rows_from(const cowa_tensor& t, int row0) {
+  cowa_tensor r = t;
+  r.ptr = static_cast<char*>(t.ptr) + (int64_t)row0 * t.stride_t * 2;
+  return r;
+}
+}  // namespace
+
+size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int max_len, int Hq, int Hkv, int d) {
+  Pat p;
+  if (check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, max_len, Hq, Hkv, d) != COWA_OK) return 0;
+  return bwd_varlen_stats_bytes(max_len, Hq, Hkv, d) + align_up((size_t)Hq * max_len * sizeof(float), 256);
+}
+
+cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, const int32_t* cu_seqlens, int total, int max_len,
+                            int Hq, int Hkv, int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+                            const float* lse, cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(1, total, Hq, Hkv, d));
+  COWA_TRY(check_heads(1, max_len, Hq, Hkv, d));
+  if (n_seq < 1 || !cu_seqlens || !lse) return COWA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0 || cu_seqlens[n_seq] != total) return COWA_ERR_INVALID_ARG;
+  for (int s = 0; s < n_seq; ++s) {
+    if (cu_seqlens[s + 1] < cu_seqlens[s]) return COWA_ERR_INVALID_ARG;
+    if (cu_seqlens[s + 1] - cu_seqlens[s] > max_len) return COWA_ERR_WORKSPACE;
+  }
+  const cowa_tensor* all[] = {&q, &k, &v, &o, &dO, &dq, &dk, &dv};
+  for (const cowa_tensor* t : all) COWA_TRY(check_tensor(*t));
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return COWA_ERR_ALIGNMENT;
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_bwd_varlen_workspace_size(pat, max_len, Hq, Hkv, d)));
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t stats = bwd_varlen_stats_bytes(max_len, Hq, Hkv, d);
+  float* lse_seq = reinterpret_cast<float*>(static_cast<char*>(ws) + stats);
+  for (int s = 0; s < n_seq; ++s) {
+    const int row0 = cu_seqlens[s], len = cu_seqlens[s + 1] - row0;
+    if (len == 0) continue;
+    // the sequence's lse rows: H_q rows of len floats, pitch total -> contiguous [H_q, len]
+    if (cudaMemcpy2DAsync(lse_seq, (size_t)len * sizeof(float), lse + row0, (size_t)total * sizeof(float),
+                          (size_t)len * sizeof(float), (size_t)Hq, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return COWA_ERR_CUDA;
+    COWA_TRY(cowa_bwd_stages(pat, 1, len, Hq, Hkv, d, rows_from(q, row0), rows_from(k, row0), rows_from(v, row0),
+                             rows_from(o, row0), lse_seq, rows_from(dO, row0), rows_from(dq, row0),
+                             rows_from(dk, row0), rows_from(dv, row0),
+                             COWA_BWD_PREPROCESS | COWA_BWD_DKDV | COWA_BWD_DQ, ws, stats, stream));
+  }
+  return COWA_OK;
+}
+
 // ------------------------------------------------------------------------------ introspection
 cowa_status cowa_visible_counts(const cowa_pattern* pat, int Hkv, int N, int64_t* out) {
   Pat p;
