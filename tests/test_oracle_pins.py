@@ -137,6 +137,25 @@ def test_swa_with_sinks_golden():
             assert got == want, t
 
 
+def test_small_cowa_layer_golden():
+    """Visible sets of a 4-head layer (S=2, L=3, T=18; D=4 and the duplicated D=2) worked out by
+    hand from the definition (golden), against the oracle's mask and the library's host counts."""
+    from structured_sparse_attention_cowa_b200 import cowa as cw
+
+    with open(os.path.join(GOLDEN, "cowa_small_visible.txt")) as f:
+        rows = [ln for ln in f if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 28
+    for line in rows:
+        head, rng = line.split(":")
+        D, t, G = (int(x) for x in head.split())
+        want = _parse_ranges(rng.strip())
+        pat = orc.Pattern(S=2, L=3, T=18, D=D)
+        got = np.nonzero(orc.visible_mask(np.array([t]), t + 1, pat, G, 4)[0])[0].tolist()
+        assert got == want, (D, t, G)
+        counts = cw.visible_counts(cw.Pattern(2, 3, 18, D), 4, 20)
+        assert counts[G, t] == len(want), (D, t, G)
+
+
 def _count_closed_form(t, S, L, lo, hi):
     """|sink U band U interval| at position t by inclusion-exclusion over three ranges."""
     def inter(*rs):
