@@ -11,7 +11,8 @@ import torch
 from oracle import cowa_oracle as orc
 from structured_sparse_attention_cowa_b200 import cowa as cw
 from structured_sparse_attention_cowa_b200 import synth
-from tests.gpu_helpers import GRAD_RTOL, DeviceView, edge_rows, host_and_device, oracle_pattern, rel_fro, to64
+from tests.gpu_helpers import (GRAD_RTOL, DeviceView, edge_rows, grad_bounds, grad_errors, host_and_device,
+                               oracle_pattern, rel_fro, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +38,9 @@ def _run(dev_inputs, pat):
 def _check_full(B, N, Hq, Hkv, d, pat, device, extra=0):
     host, dev = _inputs(B, N, Hq, Hkv, d, device, extra)
     dq, dk, dv = _run(dev, pat)
-    wq, wk, wv = orc.attention_bwd(*host, oracle_pattern(pat))
-    errs = (rel_fro(to64(dq), wq), rel_fro(to64(dk), wk), rel_fro(to64(dv), wv))
+    op = oracle_pattern(pat)
+    want = orc.attention_bwd(*host, op)
+    errs = grad_errors((to64(dq), to64(dk), to64(dv)), want, grad_bounds(*host, op.sm_scale(d)))
     assert max(errs) <= GRAD_RTOL, errs
 
 
@@ -57,6 +59,8 @@ def test_bwd_tiny_config(cuda_device, D):
     (1, 700, 8, 4, 128, cw.Pattern(32, 100, 500, 4)),        # N > T
     (1, 300, 2, 1, 128, cw.Pattern(7, 30, 300, 2, kv_head_base=1, h_kv_global=2)),  # TP rank
     (1, 256, 16, 2, 64, cw.Pattern(16, 64, 256, 2, softmax_scale=0.3)),  # group of 8
+    (2, 1, 10, 2, 128, cw.Pattern(64, 128, 1024, 2)),       # N = 1: one key per row, dq = dk = 0
+    (1, 300, 8, 4, 128, cw.Pattern(0, 1, 0, 4)),            # S = 0, L = 1, T = 0: each row sees only itself
 ])
 def test_bwd_edge_shapes(cuda_device, B, N, Hq, Hkv, d, pat):
     _check_full(B, N, Hq, Hkv, d, pat, cuda_device, extra=2)

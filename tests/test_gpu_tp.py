@@ -13,7 +13,7 @@ import torch
 from oracle import cowa_oracle as orc
 from structured_sparse_attention_cowa_b200 import cowa as cw
 from structured_sparse_attention_cowa_b200 import shard
-from tests.gpu_helpers import GRAD_RTOL, LSE_ATOL, O_ATOL, host_and_device, oracle_pattern, rel_fro, to64
+from tests.gpu_helpers import GRAD_RTOL, LSE_ATOL, O_ATOL, grad_bounds, grad_errors, host_and_device, oracle_pattern, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +46,8 @@ def test_tp_prefill_runs_reproduce_the_layer(cuda_device, P, order):
             qs, ks = slice(qh.start, qh.stop), slice(kh.start, kh.stop)
             assert np.abs(to64(o) - wo[:, :, qs]).max() <= O_ATOL, (r, run)
             assert np.abs(lse.cpu().numpy() - wl[:, qs]).max() <= LSE_ATOL, (r, run)
-            errs = (rel_fro(to64(dq), wq[:, :, qs]), rel_fro(to64(dk), wk[:, :, ks]), rel_fro(to64(dv), wv[:, :, ks]))
+            bounds = grad_bounds(q64[:, :, qs], k64[:, :, ks], v64[:, :, ks], do64[:, :, qs], op.sm_scale(d))
+            errs = grad_errors((to64(dq), to64(dk), to64(dv)), (wq[:, :, qs], wk[:, :, ks], wv[:, :, ks]), bounds)
             assert max(errs) <= GRAD_RTOL, (r, run, errs)
             covered += list(kh)
     assert sorted(covered) == list(range(Hkv))

@@ -1,8 +1,10 @@
 """GPU parity: the backward of a packed variable-length batch (cowa_bwd_varlen, host cu_seqlens)
 against the fp64 oracle's backward over each sequence alone.
 
-Tolerance: relative Frobenius error <= 1e-2 for dq, dk, dv per sequence, as for cowa_bwd.  The
-o and lse fed to the backward come from cowa_fwd_varlen on the same packed batch."""
+Tolerance: relative Frobenius error <= 1e-2 for dq, dk, dv per sequence, as for cowa_bwd; the
+length-1 sequence has dq = dk = 0 exactly and is judged by its absolute error (gpu_helpers.VANISH).
+The o and lse fed to the backward come from cowa_fwd_varlen on the same packed batch.  Every
+sequence is checked before the assertion, so a failure reports all of them."""
 
 import numpy as np
 import pytest
@@ -10,7 +12,7 @@ import torch
 
 from oracle import cowa_oracle as orc
 from structured_sparse_attention_cowa_b200 import cowa as cw
-from tests.gpu_helpers import GRAD_RTOL, host_and_device, oracle_pattern, rel_fro, to64
+from tests.gpu_helpers import GRAD_RTOL, grad_bounds, grad_errors, host_and_device, oracle_pattern, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -30,9 +32,13 @@ def test_bwd_varlen_packed_batch(cuda_device, Hq, Hkv, d, pat, lens):
     dq, dk, dv = cw.cowa_bwd_varlen(q[0], k[0], v[0], o, lse, do[0], cu, pat)
     torch.cuda.synchronize()
     op = oracle_pattern(pat)
+    report = []
     for s_, (a_, b_) in enumerate(zip(cu[:-1], cu[1:])):
         if b_ == a_:
             continue
-        wq, wk, wv = orc.attention_bwd(q64[:, a_:b_], k64[:, a_:b_], v64[:, a_:b_], do64[:, a_:b_], op)
-        errs = (rel_fro(to64(dq[a_:b_]), wq[0]), rel_fro(to64(dk[a_:b_]), wk[0]), rel_fro(to64(dv[a_:b_]), wv[0]))
-        assert max(errs) <= GRAD_RTOL, (s_, errs)
+        sl = (q64[:, a_:b_], k64[:, a_:b_], v64[:, a_:b_], do64[:, a_:b_])
+        want = [w[0] for w in orc.attention_bwd(*sl, op)]
+        got = (to64(dq[a_:b_]), to64(dk[a_:b_]), to64(dv[a_:b_]))
+        bounds = grad_bounds(*sl, op.sm_scale(d))
+        report.append((s_, b_ - a_, grad_errors(got, want, bounds)))
+    assert all(max(e) <= GRAD_RTOL for _, _, e in report), report
