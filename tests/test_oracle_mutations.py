@@ -60,7 +60,18 @@ def _bwd_dv_transposed_heads(q, k, v, do, pat):
     return dq, dk, dv[:, :, ::-1].copy()
 
 
+def _widen_shift_15(bits):
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 15).view(np.float32).astype(np.float64)
+
+
+def _widen_sign_lost(bits):
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) & 0x7FFF
+    return (b << 16).view(np.float32).astype(np.float64)
+
+
 MUTANTS = [
+    ("bf16_bits_to_f64", _widen_shift_15, [lambda: pins.test_bf16_widening_every_bit_pattern()]),
+    ("bf16_bits_to_f64", _widen_sign_lost, [lambda: pins.test_bf16_widening_every_bit_pattern()]),
     ("visible_mask", _mask_band_off_by_one, [lambda: pins.test_visible_counts_brute_force_and_closed_form(120, 5, 9, 120, 4, 4),
                                             lambda: pins.test_swa_with_sinks_golden()]),
     ("interval_of", _interval_wrong_slot, [lambda: pins.test_ablation_distinct_windows_fixed_width()]),

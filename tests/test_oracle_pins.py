@@ -384,3 +384,24 @@ def test_tile_plans_from_mask(N, BM, BN, S, L, T, H, D):
                 if j in visited:
                     assert visited[j] == all(els)
                 assert (i in bwd[(j, g)]) == (j in visited)
+
+
+def test_bf16_widening_every_bit_pattern():
+    """bf16_bits_to_f64 (how every GPU parity test hands the oracle the kernel's input bits)
+    against torch's own bf16 -> float64 conversion for all 65,536 patterns, NaNs by class, and
+    against values fixed by the bfloat16 format itself (1 sign, 8 exponent bits with bias 127,
+    7 fraction bits: the upper half of an IEEE binary32)."""
+    import torch
+
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = orc.bf16_bits_to_f64(bits)
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(want[~nan]))  # -0.0 keeps its sign
+    landmarks = {0x3F80: 1.0, 0xC000: -2.0, 0x4049: 3.140625, 0x0001: 2.0 ** -133, 0x0080: 2.0 ** -126,
+                 0x7F7F: (2 - 2.0 ** -7) * 2.0 ** 127, 0x7F80: np.inf, 0xFF80: -np.inf, 0x3E80: 0.25}
+    for b, v in landmarks.items():
+        assert orc.bf16_bits_to_f64(np.array([b], dtype=np.uint16))[0] == v, hex(b)
+    assert np.signbit(orc.bf16_bits_to_f64(np.array([0x8000], dtype=np.uint16))[0])
