@@ -27,8 +27,8 @@
  *   - Tensors are bf16 in device memory, described by cowa_tensor: a pointer
  *     plus element strides for batch, position and head; the head dimension d
  *     is contiguous.  Pointers and every stride * 2 bytes must be multiples
- *     of 16 bytes (COWA_ERR_ALIGNMENT otherwise).  d must be 64 or 128
- *     (COWA_ERR_UNSUPPORTED otherwise).
+ *     of 16 bytes (COWA_ERR_ALIGNMENT otherwise).  d must be 64 or 128 and
+ *     H_q / H_kv at most 8 (COWA_ERR_UNSUPPORTED otherwise).
  *   - The caller owns every buffer, including the workspace; the library never
  *     allocates device memory on a call.  Query the workspace size with the
  *     matching *_workspace_size function; a smaller ws_bytes returns
@@ -56,7 +56,8 @@ extern "C" {
 typedef enum {
   COWA_OK = 0,
   COWA_ERR_INVALID_ARG = 1, /* bad shape, pattern or null pointer */
-  COWA_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128} */
+  COWA_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128}, or more than 8 query heads per KV
+                               head (H_q / H_kv > 8); the E4M3-cache calls need d = 128 */
   COWA_ERR_ALIGNMENT = 3,   /* pointer or stride not 16-byte aligned */
   COWA_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
   COWA_ERR_CUDA = 5,        /* CUDA runtime/driver error at launch */
@@ -218,6 +219,44 @@ cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int H_q, int H_k
                                 const void* k_compact, const void* v_compact, const int32_t* pos, void* o,
                                 float* lse_or_null, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- decode over an E4M3 (8-bit float) cache ------------------------------------------
+ * cowa_decode with the cache stored as E4M3 codes (OCP 8-bit floating point, the E4M3FN variant:
+ * bias 7, no infinities, largest magnitude 448): the attention uses k_scale * e4m3(code) for
+ * keys and v_scale * e4m3(code) for values.  Halves the bytes a decode step reads.  Source: the
+ * decode-memory argument of "Sliding Window Attention Beats Linear Attention ...", section
+ * "Engineering Advantages" (decode throughput is set by the cache bytes read); the pages fix no
+ * cache precision, so the format, one scale per cache tensor and round-to-nearest-even saturating
+ * quantisation are this library's reading.
+ * k_cache, v_cache: uint8 codes, cowa_tensor with strides in bytes (multiples of 16); d must be
+ * 128 (COWA_ERR_UNSUPPORTED otherwise).  k_scale, v_scale finite and > 0.  q_t bf16 as for
+ * cowa_decode (used in f16 by the kernel: bf16 values of magnitude 2^-14 .. 65504 are exact in
+ * f16).  Workspace: cowa_decode_fp8_workspace_size.  Errors as for cowa_decode. */
+size_t cowa_decode_fp8_workspace_size(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap);
+cowa_status cowa_decode_fp8(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap, const void* q_t,
+                            cowa_tensor k_cache, cowa_tensor v_cache, float k_scale, float v_scale,
+                            const int32_t* pos, void* o, float* lse_or_null, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* The compacted per-head cache (see cowa_compact_build) holding E4M3 codes: build from a full
+ * E4M3 cache (uint8 cowa_tensor, byte strides), append one token's codes (k_new, v_new uint8
+ * [B, H_kv, 128] contiguous), decode with the scales of cowa_decode_fp8.  d = 128 only. */
+cowa_status cowa_compact_build_fp8(const cowa_pattern* pat, int B, int N, int H_kv, int d, cowa_tensor k,
+                                   cowa_tensor v, void* k_compact, void* v_compact, void* stream);
+cowa_status cowa_compact_append_fp8(const cowa_pattern* pat, int B, int H_kv, int d, const void* k_new,
+                                    const void* v_new, const int32_t* pos, void* k_compact, void* v_compact,
+                                    void* stream);
+size_t cowa_decode_fp8_compact_workspace_size(const cowa_pattern* pat, int B, int H_q, int H_kv, int d);
+cowa_status cowa_decode_fp8_compact(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, const void* q_t,
+                                    const void* k_compact, const void* v_compact, float k_scale, float v_scale,
+                                    const int32_t* pos, void* o, float* lse_or_null, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* E4M3 codes of x / scale for n bf16 elements (device pointers; n a multiple of 8; x 16-byte and
+ * codes 8-byte aligned): a float32 multiply by the float32 reciprocal of scale, then round to
+ * nearest even, saturating at +-448.  Stream-ordered; COWA_ERR_INVALID_ARG / COWA_ERR_ALIGNMENT
+ * before any launch. */
+cowa_status cowa_quantize_e4m3(const void* x, void* codes, int64_t n, float scale, void* stream);
+
 /* ---- decode without a caller workspace -----------------------------------------------------
  * This entry point has no counterpart on the CoWA pages; it is a convenience of this library for
  * callers that cannot allocate device memory (runtimes that reserve the whole memory pool up
@@ -230,19 +269,26 @@ cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int H_q, int H_k
  * until the process exits.  The call allocates nothing (no cudaMalloc, no allocating library
  * routine).
  *   - The first call made with a given device current looks up the scratch address on that
- *     device (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     device (cudaGetSymbolAddress); make that first call before any stream capture.  The
+ *     lookup is repeated only if the device's context has been replaced since (after a
+ *     cudaDeviceReset the library's device variables live at new addresses).
  *   - Every call shares the one scratch array of its device and leaves its contents behind.
  *     The status word is cleared at the start of each call.  Calls that overlap on the GPU
  *     (e.g. on two streams without ordering between them) race on the scratch and give
  *     undefined results: order them on one stream or synchronize between them.
  *   - A configuration whose workspace (cowa_decode_workspace_size) exceeds the scratch size
  *     returns COWA_ERR_WORKSPACE without launching.  Other argument errors are those of
- *     cowa_decode.  A device-side timeout leaves its status in the library's scratch, which the
- *     caller cannot read: use cowa_decode when the status matters. */
+ *     cowa_decode.  A device-side timeout leaves its status in the library's scratch; read it
+ *     with cowa_decode_noalloc_status. */
 #define COWA_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 cowa_status cowa_decode_noalloc(const cowa_pattern* pat, int B, int H_q, int H_kv, int d, int T_cap,
                                 const void* q_t, cowa_tensor k_cache, cowa_tensor v_cache,
                                 const int32_t* pos, void* o, float* lse_or_null, void* stream);
+/* Synchronizes `stream`, then reads and clears the status word in the current device's
+ * cowa_decode_noalloc scratch: COWA_OK, or COWA_ERR_TIMEOUT if a bounded device wait of an
+ * earlier cowa_decode_noalloc call on this device ran out (COWA_ERR_CUDA if the stream failed).
+ * Copies 4 bytes to the host and allocates nothing. */
+cowa_status cowa_decode_noalloc_status(void* stream);
 
 /* ---- status --------------------------------------------------------------------------------
  * Synchronizes `stream`, reads and clears the device status word in `ws` (the workspace of an

@@ -14,7 +14,9 @@ acceptable (a workspace the binding allocates itself is not checked).
 
 Function names follow the C ABI (include/cowa.h): cowa_fwd, cowa_fwd_chunk,
 cowa_fwd_varlen, cowa_bwd, cowa_bwd_varlen, cowa_decode, cowa_decode_compact (with compact_cache /
-compact_append), cowa_decode_noalloc, plus the planner introspection helpers.
+compact_append), the E4M3-cache decodes (cowa_decode_fp8, cowa_decode_fp8_compact, with
+quantize_e4m3, compact_cache_fp8, compact_append_fp8), cowa_decode_noalloc, plus the planner
+introspection helpers.
 """
 
 from __future__ import annotations
@@ -107,6 +109,8 @@ def lib() -> ctypes.CDLL:
     L.cowa_decode.restype = i
     L.cowa_decode_noalloc.argtypes = [P, i, i, i, i, i, vp, T, T, vp, vp, vp, vp]
     L.cowa_decode_noalloc.restype = i
+    L.cowa_decode_noalloc_status.argtypes = [vp]
+    L.cowa_decode_noalloc_status.restype = i
     L.cowa_compact_rows.argtypes = [P, i]
     L.cowa_compact_rows.restype = i
     L.cowa_compact_build.argtypes = [P, i, i, i, i, T, T, vp, vp, vp]
@@ -117,6 +121,21 @@ def lib() -> ctypes.CDLL:
     L.cowa_decode_compact_workspace_size.restype = sz
     L.cowa_decode_compact.argtypes = [P, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.cowa_decode_compact.restype = i
+    f = ctypes.c_float
+    L.cowa_decode_fp8_workspace_size.argtypes = [P, i, i, i, i, i]
+    L.cowa_decode_fp8_workspace_size.restype = sz
+    L.cowa_decode_fp8.argtypes = [P, i, i, i, i, i, vp, T, T, f, f, vp, vp, vp, vp, sz, vp]
+    L.cowa_decode_fp8.restype = i
+    L.cowa_quantize_e4m3.argtypes = [vp, vp, ctypes.c_int64, f, vp]
+    L.cowa_quantize_e4m3.restype = i
+    L.cowa_compact_build_fp8.argtypes = [P, i, i, i, i, T, T, vp, vp, vp]
+    L.cowa_compact_build_fp8.restype = i
+    L.cowa_compact_append_fp8.argtypes = [P, i, i, i, vp, vp, vp, vp, vp, vp]
+    L.cowa_compact_append_fp8.restype = i
+    L.cowa_decode_fp8_compact_workspace_size.argtypes = [P, i, i, i, i]
+    L.cowa_decode_fp8_compact_workspace_size.restype = sz
+    L.cowa_decode_fp8_compact.argtypes = [P, i, i, i, i, vp, vp, vp, f, f, vp, vp, vp, vp, sz, vp]
+    L.cowa_decode_fp8_compact.restype = i
     L.cowa_workspace_status.argtypes = [vp, vp]
     L.cowa_workspace_status.restype = i
     L.cowa_status_string.argtypes = [i]
@@ -444,6 +463,126 @@ def cowa_decode_noalloc(q_t, k_cache, v_cache, pos, pattern: Pattern, out, lse=N
         _cache_tensor(v_cache, layout), pos.data_ptr(), out.data_ptr(),
         lse.data_ptr() if lse is not None else None, _stream(stream)))
     return out, lse
+
+
+# ---------------------------------------------------------------------------- E4M3 cache
+def _u8_cuda(name, x):
+    import torch
+
+    if not (x.is_cuda and x.dtype == torch.uint8):
+        raise TypeError(f"{name} must be a CUDA uint8 tensor of E4M3 codes")
+
+
+def quantize_e4m3(x, scale: float, out=None, stream=None):
+    """E4M3 codes (uint8, same shape) of the bf16 tensor x divided by scale: a float32 multiply by
+    the float32 reciprocal of scale, round to nearest even, saturating at +-448."""
+    import torch
+
+    _bf16_cuda("x", x)
+    if not x.is_contiguous() or x.numel() % 8 != 0:
+        raise ValueError("x must be contiguous with a multiple of 8 elements")
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    _check("cowa_quantize_e4m3", lib().cowa_quantize_e4m3(x.data_ptr(), out.data_ptr(), x.numel(), float(scale),
+                                                          _stream(stream)))
+    return out
+
+
+def cowa_decode_fp8(q_t, k_codes, v_codes, pos, pattern: Pattern, k_scale: float, v_scale: float,
+                    layout: str = "bhtd", out=None, lse=None, workspace=None, stream=None):
+    """cowa_decode over an E4M3 cache: keys k_scale * e4m3(k_codes), values v_scale * e4m3(v_codes);
+    codes uint8 [B, H_kv, T_cap, 128] ("bhtd") or [B, T_cap, H_kv, 128] ("bthd")."""
+    import torch
+
+    _bf16_cuda("q_t", q_t)
+    _u8_cuda("k_codes", k_codes)
+    _u8_cuda("v_codes", v_codes)
+    if not q_t.is_contiguous():
+        raise ValueError("q_t must be contiguous [B, H_q, d]")
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise TypeError("pos must be a CUDA int32 tensor [B]")
+    B, Hq, d = q_t.shape
+    Hkv, T_cap = (k_codes.shape[1], k_codes.shape[2]) if layout == "bhtd" else (k_codes.shape[2], k_codes.shape[1])
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_t.device) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q_t.device) if lse is None else lse
+    pat = pattern.c()
+    L = lib()
+    if workspace is None:
+        workspace = _workspace(L.cowa_decode_fp8_workspace_size(ctypes.byref(pat), B, Hq, Hkv, d, T_cap), q_t.device)
+    _check("cowa_decode_fp8", L.cowa_decode_fp8(ctypes.byref(pat), B, Hq, Hkv, d, T_cap, q_t.data_ptr(),
+                                                _cache_tensor(k_codes, layout), _cache_tensor(v_codes, layout),
+                                                float(k_scale), float(v_scale), pos.data_ptr(), out.data_ptr(),
+                                                lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                                _stream(stream)))
+    return out, lse
+
+
+def compact_cache_fp8(k_codes, v_codes, pattern: Pattern, out=None, stream=None):
+    """Compacted E4M3 caches [B, H_kv, rows, 128] (uint8) built from codes [B, N, H_kv, 128]."""
+    import torch
+
+    _u8_cuda("k_codes", k_codes)
+    _u8_cuda("v_codes", v_codes)
+    B, N, Hkv, d = k_codes.shape
+    rows = compact_rows(pattern, Hkv)
+    if out is None:
+        out = (torch.zeros((B, Hkv, rows, d), dtype=torch.uint8, device=k_codes.device),
+               torch.zeros((B, Hkv, rows, d), dtype=torch.uint8, device=k_codes.device))
+    kc, vc = out
+    _check("cowa_compact_build_fp8", lib().cowa_compact_build_fp8(ctypes.byref(pattern.c()), B, N, Hkv, d,
+                                                                  _t4(k_codes), _t4(v_codes), kc.data_ptr(),
+                                                                  vc.data_ptr(), _stream(stream)))
+    return kc, vc
+
+
+def compact_append_fp8(kc, vc, k_new, v_new, pos, pattern: Pattern, stream=None):
+    """Appends one token's codes (k_new, v_new uint8 [B, H_kv, 128]) at pos[b] to compacted E4M3 caches."""
+    import torch
+
+    _u8_cuda("k_new", k_new)
+    _u8_cuda("v_new", v_new)
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise ValueError("pos must be a CUDA int32 tensor")
+    B, Hkv, _, d = kc.shape
+    k_new, v_new = k_new.contiguous(), v_new.contiguous()
+    _check("cowa_compact_append_fp8", lib().cowa_compact_append_fp8(ctypes.byref(pattern.c()), B, Hkv, d,
+                                                                    k_new.data_ptr(), v_new.data_ptr(), pos.data_ptr(),
+                                                                    kc.data_ptr(), vc.data_ptr(), _stream(stream)))
+
+
+def cowa_decode_fp8_compact(q_t, kc, vc, pos, pattern: Pattern, k_scale: float, v_scale: float, out=None,
+                            lse=None, workspace=None, stream=None):
+    """cowa_decode_fp8 over compacted E4M3 caches kc, vc [B, H_kv, rows, 128] (uint8)."""
+    import torch
+
+    _bf16_cuda("q_t", q_t)
+    _u8_cuda("k_compact", kc)
+    _u8_cuda("v_compact", vc)
+    if not (q_t.is_contiguous() and kc.is_contiguous() and vc.is_contiguous()):
+        raise ValueError("q_t and the compacted caches must be contiguous")
+    if pos.dtype != torch.int32 or not pos.is_cuda:
+        raise ValueError("pos must be a CUDA int32 tensor")
+    B, Hq, d = q_t.shape
+    Hkv = kc.shape[1]
+    if kc.shape[2] != compact_rows(pattern, Hkv):
+        raise ValueError("compacted cache has the wrong number of rows for this pattern")
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_t.device) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q_t.device) if lse is None else lse
+    pat = pattern.c()
+    L = lib()
+    if workspace is None:
+        workspace = _workspace(L.cowa_decode_fp8_compact_workspace_size(ctypes.byref(pat), B, Hq, Hkv, d), q_t.device)
+    _check("cowa_decode_fp8_compact", L.cowa_decode_fp8_compact(ctypes.byref(pat), B, Hq, Hkv, d, q_t.data_ptr(),
+                                                                kc.data_ptr(), vc.data_ptr(), float(k_scale),
+                                                                float(v_scale), pos.data_ptr(), out.data_ptr(),
+                                                                lse.data_ptr(), workspace.data_ptr(),
+                                                                workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def decode_noalloc_status(stream=None) -> int:
+    """Synchronize the stream, read (and clear) the status word of cowa_decode_noalloc's scratch
+    on the current device; returns the cowa_status code."""
+    return lib().cowa_decode_noalloc_status(_stream(stream))
 
 
 def workspace_status(workspace, stream=None) -> int:

@@ -92,6 +92,30 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int d, int n_t, int n_h,
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8(CUtensorMap* map, const void* base, int d, int n_t, int n_h, int n_b, int64_t stride_t,
+                  int64_t stride_h, int64_t stride_b, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n_t, (cuuint64_t)n_h, (cuuint64_t)n_b};
+  cuuint64_t strides[3] = {(cuuint64_t)stride_t, (cuuint64_t)stride_h, (cuuint64_t)stride_b};
+  cuuint32_t box[4] = {128, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+// a tensor of one-byte elements: pointer and byte strides multiples of 16
+cowa_status check_tensor8(const cowa_tensor& t) {
+  if (!t.ptr) return COWA_ERR_INVALID_ARG;
+  auto ok = [](int64_t v) { return v > 0 && v % 16 == 0; };
+  if (!aligned16(t.ptr) || !ok(t.stride_t) || !ok(t.stride_h) || !ok(t.stride_b)) return COWA_ERR_ALIGNMENT;
+  return COWA_OK;
+}
+}  // namespace
+
 }  // namespace cowa
 
 using namespace cowa;
@@ -254,6 +278,131 @@ cowa_status cowa_decode(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, 
                       v_cache.stride_b, 64))
     return COWA_ERR_CUDA;
   return launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------ E4M3 cache
+size_t cowa_decode_fp8_workspace_size(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, int T_cap) {
+  return d == 128 ? cowa_decode_workspace_size(pat, B, Hq, Hkv, d, T_cap) : 0;
+}
+
+cowa_status cowa_decode_fp8(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, int T_cap, const void* q_t,
+                            cowa_tensor k_cache, cowa_tensor v_cache, float k_scale, float v_scale,
+                            const int32_t* pos, void* o, float* lse_or_null, void* ws, size_t ws_bytes,
+                            void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, 1, Hq, Hkv, d));
+  if (d != 128) return COWA_ERR_UNSUPPORTED;
+  if (T_cap < 1 || !q_t || !pos || !o || !(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) ||
+      !isfinite(v_scale))
+    return COWA_ERR_INVALID_ARG;
+  COWA_TRY(check_tensor8(k_cache));
+  COWA_TRY(check_tensor8(v_cache));
+  if (!aligned16(q_t) || !aligned16(o) || (lse_or_null && (reinterpret_cast<uintptr_t>(lse_or_null) & 3u)))
+    return COWA_ERR_ALIGNMENT;
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_decode_fp8_workspace_size(pat, B, Hq, Hkv, d, T_cap)));
+
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.pat = p; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.T_cap = T_cap;
+  a.q_t = q_t; a.pos = pos; a.o = o; a.lse = lse_or_null;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.chunk = decode_chunk_tokens(p, B, Hkv, T_cap);
+  a.n_split = decode_num_splits(p, T_cap, a.chunk);
+  a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f * k_scale;
+  a.kv8 = 1;
+  a.v_scale = v_scale;
+  if (!make_tmap_u8(&a.tm_k, k_cache.ptr, d, T_cap, Hkv, B, k_cache.stride_t, k_cache.stride_h, k_cache.stride_b,
+                    64) ||
+      !make_tmap_u8(&a.tm_v, v_cache.ptr, d, T_cap, Hkv, B, v_cache.stride_t, v_cache.stride_h, v_cache.stride_b,
+                    64))
+    return COWA_ERR_CUDA;
+  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+}
+
+// compacted E4M3 cache: rows of d = 128 codes (128 bytes, the row size of a d = 64 bf16 cache, so
+// the row-copy kernels of the bf16 cache serve it with strides counted in 2-byte units)
+cowa_status cowa_compact_build_fp8(const cowa_pattern* pat, int B, int N, int Hkv, int d, cowa_tensor k,
+                                   cowa_tensor v, void* k_compact, void* v_compact, void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, N, Hkv, Hkv, d));
+  if (d != 128) return COWA_ERR_UNSUPPORTED;
+  COWA_TRY(check_tensor8(k));
+  COWA_TRY(check_tensor8(v));
+  if (!k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(k_compact) || !aligned16(v_compact)) return COWA_ERR_ALIGNMENT;
+  return launch_compact_build(p, B, N, Hkv, 64, k.ptr, k.stride_b / 2, k.stride_t / 2, k.stride_h / 2, v.ptr,
+                              v.stride_b / 2, v.stride_t / 2, v.stride_h / 2, k_compact, v_compact,
+                              reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
+}
+
+cowa_status cowa_compact_append_fp8(const cowa_pattern* pat, int B, int Hkv, int d, const void* k_new,
+                                    const void* v_new, const int32_t* pos, void* k_compact, void* v_compact,
+                                    void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, 1, Hkv, Hkv, d));
+  if (d != 128) return COWA_ERR_UNSUPPORTED;
+  if (!k_new || !v_new || !pos || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_compact) || !aligned16(v_compact))
+    return COWA_ERR_ALIGNMENT;
+  return launch_compact_append(p, B, Hkv, 64, k_new, v_new, pos, k_compact, v_compact,
+                               reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
+}
+
+size_t cowa_decode_fp8_compact_workspace_size(const cowa_pattern* pat, int B, int Hq, int Hkv, int d) {
+  return d == 128 ? cowa_decode_compact_workspace_size(pat, B, Hq, Hkv, d) : 0;
+}
+
+cowa_status cowa_decode_fp8_compact(const cowa_pattern* pat, int B, int Hq, int Hkv, int d, const void* q_t,
+                                    const void* k_compact, const void* v_compact, float k_scale, float v_scale,
+                                    const int32_t* pos, void* o, float* lse_or_null, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  Pat p;
+  COWA_TRY(check_pattern(pat, Hkv, &p));
+  COWA_TRY(check_heads(B, 1, Hq, Hkv, d));
+  if (d != 128) return COWA_ERR_UNSUPPORTED;
+  if (!q_t || !pos || !o || !k_compact || !v_compact || !(k_scale > 0.f) || !(v_scale > 0.f) ||
+      !isfinite(k_scale) || !isfinite(v_scale))
+    return COWA_ERR_INVALID_ARG;
+  if (!aligned16(q_t) || !aligned16(o) || !aligned16(k_compact) || !aligned16(v_compact) ||
+      (lse_or_null && (reinterpret_cast<uintptr_t>(lse_or_null) & 3u)))
+    return COWA_ERR_ALIGNMENT;
+  COWA_TRY(check_ws(ws, ws_bytes, cowa_decode_fp8_compact_workspace_size(pat, B, Hq, Hkv, d)));
+
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.pat = p; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.T_cap = kCompactSpan;
+  a.q_t = q_t; a.pos = pos; a.o = o; a.lse = lse_or_null;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.partials = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.chunk = decode_chunk_tokens(p, B, Hkv, kCompactSpan);
+  a.n_split = decode_num_splits(p, kCompactSpan, a.chunk, true);
+  a.scale_log2 = scale_of(pat, d) * 1.4426950408889634f * k_scale;
+  a.compact = 1;
+  a.cg = compact_geom(p);
+  a.kv8 = 1;
+  a.v_scale = v_scale;
+  const int64_t rows = a.cg.rows;
+  if (!make_tmap_u8(&a.tm_k, k_compact, d, (int)rows, Hkv, B, d, rows * d, (int64_t)Hkv * rows * d, 64) ||
+      !make_tmap_u8(&a.tm_v, v_compact, d, (int)rows, Hkv, B, d, rows * d, (int64_t)Hkv * rows * d, 64))
+    return COWA_ERR_CUDA;
+  return launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? COWA_OK : COWA_ERR_CUDA;
+}
+
+cowa_status cowa_quantize_e4m3(const void* x, void* codes, int64_t n, float scale, void* stream) {
+  if (!x || !codes || n < 0 || n % 8 != 0 || !(scale > 0.f) || !isfinite(scale)) return COWA_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 7u)) return COWA_ERR_ALIGNMENT;
+  const float inv = 1.0f / scale;
+  return launch_quantize_e4m3(x, codes, n, inv, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? COWA_OK
+             : COWA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------------ forward

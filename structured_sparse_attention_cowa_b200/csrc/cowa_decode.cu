@@ -36,17 +36,70 @@ namespace {
 constexpr int kDecWarps = 4;                        // compute warps per CTA
 constexpr int kDecThreads = (kDecWarps + 1) * 32;   // + one TMA producer warp
 constexpr int kSubTok = 64;                         // tokens per sub-tile (TMA box rows)
-constexpr int kStages = 3;                          // sub-tile ring depth
+constexpr int kStages = 3;                          // sub-tile ring depth (bf16 cache)
+constexpr int kMaxStages = 4;                       // ring depth of the E4M3 cache (half-size stages)
 constexpr int kBoxBytes = kSubTok * 128;            // one [64 rows x 64 bf16] box
 constexpr float kDecRescale = 8.0f;                 // lazy-rescale threshold, log2 units
 
-template <int D>
+// KV8: the cache holds E4M3 codes (one byte per element) instead of bf16; each compute warp
+// widens its 16 token rows of a sub-tile to f16 in a scratch tile of its own and runs the same
+// MMAs in f16 (E4M3 values are exact in f16).
+template <int D, bool KV8 = false>
 struct DecGeom {
-  static constexpr int kUnits = D / 64;                  // boxes per row
-  static constexpr int kTileBytes = kUnits * kBoxBytes;  // K (or V) sub-tile
+  static_assert(!KV8 || D == 128, "the E4M3 cache needs whole 128-byte rows (d = 128)");
+  static constexpr int kUnits = KV8 ? 1 : D / 64;          // 128-byte TMA boxes per row
+  static constexpr int kBoxElems = KV8 ? 128 : 64;         // elements per box row
+  static constexpr int kTileBytes = kUnits * kBoxBytes;    // K (or V) sub-tile as stored
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+  static constexpr int kStages = KV8 ? kMaxStages : ::cowa::kStages;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kWarpScratch = KV8 ? 2 * (D / 64) * 16 * 128 : 0;  // f16 K and V, 16 rows
+  static constexpr int kSmemBytes = kRingBytes + kDecWarps * kWarpScratch + 1024;
 };
+
+// shared address of 16-byte unit u (8 halves: d = 8u..8u+7) of row r of a 16-row f16 tile in the
+// same swizzled form as a TMA tile (128-byte rows, 16-row boxes of 64 halves)
+__device__ __forceinline__ uint32_t unit_addr16(uint32_t tile, int r, int u) {
+  return tile + (u >> 3) * (16 * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  // the low byte becomes the low half
+  uint32_t r;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(r) : "r"(two_codes));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));  // first source -> upper half
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void mma_16816_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
 
 // shared address of 16-byte unit u (d elements 8u..8u+7) of token row r of a swizzled tile
 __device__ __forceinline__ uint32_t unit_addr(uint32_t tile, int r, int u) {
@@ -58,16 +111,17 @@ __device__ __forceinline__ float safe_ex2_diff(float a, float m) {
   return a == -INFINITY ? 0.f : ptx::ex2(a - m);
 }
 
-template <int GRP, int D>
+template <int GRP, int D, bool KV8>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   static_assert(GRP >= 1 && GRP <= 8, "query heads per KV head must fit the MMA's first 8 rows");
-  using Geo = DecGeom<D>;
+  using Geo = DecGeom<D, KV8>;
   constexpr int KS = D / 16;  // k-steps of the score MMA
   constexpr int NT = D / 8;   // n-tiles of the P.V MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  constexpr int kStages = Geo::kStages;
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
   __shared__ int abort_flag;
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -151,8 +205,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         const int row = cache_row(p_base + st * kSubTok);
 #pragma unroll
         for (int u = 0; u < Geo::kUnits; ++u) {
-          ptx::tma_load_4d(ks + u * kBoxBytes, &a.tm_k, &full_bar[s], u * 64, row, g, b);
-          ptx::tma_load_4d(vs + u * kBoxBytes, &a.tm_v, &full_bar[s], u * 64, row, g, b);
+          ptx::tma_load_4d(ks + u * kBoxBytes, &a.tm_k, &full_bar[s], u * Geo::kBoxElems, row, g, b);
+          ptx::tma_load_4d(vs + u * kBoxBytes, &a.tm_v, &full_bar[s], u * Geo::kBoxElems, row, g, b);
         }
         issued = st + 1;
       }
@@ -175,8 +229,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     for (int kk = 0; kk < KS; ++kk) {
       qa[kk][0] = gr < GRP ? qrow[8 * kk + tq] : 0u;
       qa[kk][1] = gr < GRP ? qrow[8 * kk + 4 + tq] : 0u;
+      if constexpr (KV8) {  // f16 operands (bf16 values of the usual range are exact in f16)
+        qa[kk][0] = bf16x2_to_f16x2(qa[kk][0]);
+        qa[kk][1] = bf16x2_to_f16x2(qa[kk][1]);
+      }
     }
   }
+  // this warp's f16 scratch tiles (E4M3 cache only)
+  const uint32_t ksc = ptx::smem_u32(smem) + Geo::kRingBytes + warp * Geo::kWarpScratch;
+  const uint32_t vsc = ksc + Geo::kWarpScratch / 2;
   float acc[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -190,6 +251,24 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     if (!ptx::mbar_wait_warp(&full_bar[s], (st / kStages) & 1, &abort_flag, a.status)) { ok = false; break; }
     const uint32_t kt = smem_base + s * Geo::kStageBytes;
     const uint32_t vt = kt + Geo::kTileBytes;
+    if constexpr (KV8) {
+      // widen this warp's 16 rows of the E4M3 K and V sub-tiles (128-byte swizzled rows, unit u =
+      // codes of d = 16u..16u+15) to f16 (units 2u, 2u+1 of the scratch row); then the stage is free
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int x = it * 32 + lane;          // 0..255: {K, V} x 16 rows x 8 units
+        const int which = x >> 7, r = (x >> 3) & 15, u = x & 7;
+        const int rr = row0 + r;
+        const uint4 raw = lds128((which ? vt : kt) + rr * 128 + ((u ^ (rr & 7)) << 4));
+        const uint32_t dst = which ? vsc : ksc;
+        sts128(unit_addr16(dst, r, 2 * u), e4m3x2_to_f16x2(raw.x & 0xffffu), e4m3x2_to_f16x2(raw.x >> 16),
+               e4m3x2_to_f16x2(raw.y & 0xffffu), e4m3x2_to_f16x2(raw.y >> 16));
+        sts128(unit_addr16(dst, r, 2 * u + 1), e4m3x2_to_f16x2(raw.z & 0xffffu), e4m3x2_to_f16x2(raw.z >> 16),
+               e4m3x2_to_f16x2(raw.w & 0xffffu), e4m3x2_to_f16x2(raw.w >> 16));
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
+    }
     // ---- scores S[head][token] for two 8-token n-tiles
     float sc[2][4];
 #pragma unroll
@@ -198,11 +277,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 #pragma unroll
       for (int k2 = 0; k2 < KS / 2; ++k2) {
         uint32_t bb[4];
-        ptx::ldsm_x4(unit_addr(kt, row0 + 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
         const uint32_t a0[4] = {qa[2 * k2][0], 0u, qa[2 * k2][1], 0u};
         const uint32_t a1[4] = {qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u};
-        ptx::mma_16816(sc[nt], a0, bb[0], bb[1]);
-        ptx::mma_16816(sc[nt], a1, bb[2], bb[3]);
+        if constexpr (KV8) {
+          ptx::ldsm_x4(unit_addr16(ksc, 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
+          mma_16816_f16(sc[nt], a0, bb[0], bb[1]);
+          mma_16816_f16(sc[nt], a1, bb[2], bb[3]);
+        } else {
+          ptx::ldsm_x4(unit_addr(kt, row0 + 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
+          ptx::mma_16816(sc[nt], a0, bb[0], bb[1]);
+          ptx::mma_16816(sc[nt], a1, bb[2], bb[3]);
+        }
       }
     }
     // ---- online softmax (log2 domain) over this warp's 16 tokens
@@ -232,17 +317,29 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
       lsum += p[e];
     }
     // P as the A operand: tokens 2tq, 2tq+1 (first n-tile) and 8+2tq, 9+2tq (second)
-    const uint32_t pa[4] = {ptx::pack_bf16(p[0], p[1]), 0u, ptx::pack_bf16(p[2], p[3]), 0u};
+    uint32_t pa[4];
+    if constexpr (KV8) {
+      pa[0] = pack_f16(p[0], p[1]); pa[2] = pack_f16(p[2], p[3]);
+    } else {
+      pa[0] = ptx::pack_bf16(p[0], p[1]); pa[2] = ptx::pack_bf16(p[2], p[3]);
+    }
+    pa[1] = pa[3] = 0u;
     // ---- O[head][d] += P[head][token] V[token][d]
 #pragma unroll
     for (int np = 0; np < NT / 2; ++np) {
       uint32_t bb[4];
-      ptx::ldsm_x4_trans(unit_addr(vt, row0 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
-      ptx::mma_16816(acc[2 * np], pa, bb[0], bb[1]);
-      ptx::mma_16816(acc[2 * np + 1], pa, bb[2], bb[3]);
+      if constexpr (KV8) {
+        ptx::ldsm_x4_trans(unit_addr16(vsc, (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
+        mma_16816_f16(acc[2 * np], pa, bb[0], bb[1]);
+        mma_16816_f16(acc[2 * np + 1], pa, bb[2], bb[3]);
+      } else {
+        ptx::ldsm_x4_trans(unit_addr(vt, row0 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
+        ptx::mma_16816(acc[2 * np], pa, bb[0], bb[1]);
+        ptx::mma_16816(acc[2 * np + 1], pa, bb[2], bb[3]);
+      }
     }
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
+    __syncwarp();  // (KV8: the scratch is rewritten by the next sub-tile's widening)
+    if (!KV8 && lane == 0) ptx::mbar_arrive(&empty_bar[s]);
   }
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
@@ -276,7 +373,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     }
     const int h = g * GRP + hh;
     float* out = a.partials + (((size_t)b * a.Hq + h) * a.n_split + split) * (D + 2);
-    out[2 + dc] = o;
+    out[2 + dc] = KV8 ? o * a.v_scale : o;
     if (dc == 0) { out[0] = mxw; out[1] = ll; }
   }
 }
@@ -365,10 +462,10 @@ __global__ void __launch_bounds__(128) compact_build_kernel(Pat pat, CompactGeom
   }
 }
 
-template <int GRP, int D>
+template <int GRP, int D, bool KV8>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-  using Geo = DecGeom<D>;
-  auto kern = decode_split_kernel<GRP, D>;
+  using Geo = DecGeom<D, KV8>;
+  auto kern = decode_split_kernel<GRP, D, KV8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_split, a.Hkv, a.B);
@@ -380,17 +477,17 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool KV8 = false>
 cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
   switch (a.Hq / a.Hkv) {
-    case 1: return launch_decode_t<1, D>(a, s);
-    case 2: return launch_decode_t<2, D>(a, s);
-    case 3: return launch_decode_t<3, D>(a, s);
-    case 4: return launch_decode_t<4, D>(a, s);
-    case 5: return launch_decode_t<5, D>(a, s);
-    case 6: return launch_decode_t<6, D>(a, s);
-    case 7: return launch_decode_t<7, D>(a, s);
-    case 8: return launch_decode_t<8, D>(a, s);
+    case 1: return launch_decode_t<1, D, KV8>(a, s);
+    case 2: return launch_decode_t<2, D, KV8>(a, s);
+    case 3: return launch_decode_t<3, D, KV8>(a, s);
+    case 4: return launch_decode_t<4, D, KV8>(a, s);
+    case 5: return launch_decode_t<5, D, KV8>(a, s);
+    case 6: return launch_decode_t<6, D, KV8>(a, s);
+    case 7: return launch_decode_t<7, D, KV8>(a, s);
+    case 8: return launch_decode_t<8, D, KV8>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -466,9 +563,48 @@ cudaError_t launch_compact_build(const Pat& p, int B, int N, int Hkv, int d, con
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+  if (a.kv8) return a.d == 128 ? launch_decode_d<128, true>(a, s) : cudaErrorInvalidValue;
   if (a.d == 64) return launch_decode_d<64>(a, s);
   if (a.d == 128) return launch_decode_d<128>(a, s);
   return cudaErrorInvalidValue;
+}
+
+// E4M3 codes of x * inv_scale (bf16 in, round to nearest even, saturating at +-448); n elements,
+// n even.  One thread per 8 elements.
+__global__ void quantize_e4m3_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, int64_t n8, float inv_scale) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 v = x[i];
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    uint32_t lo16, hi16;
+    {
+      const float f0 = __uint_as_float(w[2 * j] << 16) * inv_scale;
+      const float f1 = __uint_as_float(w[2 * j] & 0xffff0000u) * inv_scale;
+      uint16_t c;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(f1), "f"(f0));  // first source -> upper byte
+      lo16 = c;
+    }
+    {
+      const float f0 = __uint_as_float(w[2 * j + 1] << 16) * inv_scale;
+      const float f1 = __uint_as_float(w[2 * j + 1] & 0xffff0000u) * inv_scale;
+      uint16_t c;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(f1), "f"(f0));
+      hi16 = c;
+    }
+    out[j] = lo16 | (hi16 << 16);
+  }
+  q[i] = make_uint2(out[0], out[1]);
+}
+
+cudaError_t launch_quantize_e4m3(const void* x, void* q, int64_t n, float inv_scale, cudaStream_t s) {
+  const int64_t n8 = n / 8;
+  if (n8 > 0)
+    quantize_e4m3_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(static_cast<const uint4*>(x),
+                                                                     static_cast<uint2*>(q), n8, inv_scale);
+  return cudaGetLastError();
 }
 
 }  // namespace cowa

@@ -49,11 +49,16 @@ struct DecodeArgs {
   // compacted cache (tm_k / tm_v over [B, H_kv, rows, d]): 0 = full cache indexed by position
   int compact;
   CompactGeom cg;
+  // E4M3 cache (tm_k / tm_v over uint8 codes): scale_log2 then includes k_scale, and the
+  // partial outputs are multiplied by v_scale
+  int kv8;
+  float v_scale;
   CUtensorMap tm_k, tm_v;
 };
 int decode_chunk_tokens(const Pat& p, int B, int Hkv, int T_cap);
 int decode_num_splits(const Pat& p, int T_cap, int chunk, bool compact = false);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_quantize_e4m3(const void* x, void* q, int64_t n, float inv_scale, cudaStream_t s);
 cudaError_t launch_compact_append(const Pat& p, int B, int Hkv, int d, const void* k_new, const void* v_new,
                                   const int32_t* pos, void* kc, void* vc, cudaStream_t s);
 cudaError_t launch_compact_build(const Pat& p, int B, int N, int Hkv, int d, const void* k, int64_t ksb, int64_t kst,
