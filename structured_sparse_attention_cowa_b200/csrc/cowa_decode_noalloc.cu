@@ -10,9 +10,11 @@
 // passes every input and output buffer.
 //
 // Nothing here allocates: the scratch address of each device is looked up once (on the
-// first call made with that device current) with cudaGetSymbolAddress, the status word is
+// first call made with that device current, and again only after that device's context has
+// been replaced, e.g. by cudaDeviceReset) with cudaGetSymbolAddress, the status word is
 // cleared with an asynchronous memset on the caller's stream, and the ordinary decode path
 // runs with the scratch array as its workspace.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -28,19 +30,52 @@ static __device__ __align__(256) unsigned char g_decode_scratch[COWA_DECODE_NOAL
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};  // device address of g_decode_scratch, per device ordinal
+struct ScratchAddr {
+  void* ptr = nullptr;             // device address of g_decode_scratch
+  unsigned long long ctx_id = 0;   // the context it was looked up in
+};
+ScratchAddr g_scratch_addr[kMaxDevices];  // per device ordinal
 
-// Device address of the scratch array on the current device; looked up on first use.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+void* driver_entry(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
+// Unique id of the calling thread's current context (0 if there is none).  A device reset
+// destroys the context the scratch address was looked up in; the library's device code is
+// loaded again in the next context, possibly at another address, so the address is only
+// reused while the context is the same one.
+unsigned long long current_ctx_id() {
+  static const CtxGetCurrentFn get_cur = reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+  static const CtxGetIdFn get_id = reinterpret_cast<CtxGetIdFn>(driver_entry("cuCtxGetId"));
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device: looked up once per device (and
+// again only if that device's context has changed since).
 cowa_status scratch_on_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return COWA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchAddr& e = g_scratch_addr[dev];
+  unsigned long long id = current_ctx_id();
+  if (e.ptr == nullptr || id == 0 || id != e.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return COWA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if (id == 0) id = current_ctx_id();  // the lookup made the device's primary context current
+    e.ptr = p;
+    e.ctx_id = id;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.ptr;
   return COWA_OK;
 }
 
@@ -66,4 +101,11 @@ extern "C" cowa_status cowa_decode_noalloc(const cowa_pattern* pat, int B, int H
     return COWA_ERR_CUDA;
   return cowa_decode(pat, B, H_q, H_kv, d, T_cap, q_t, k_cache, v_cache, pos, o, lse_or_null, scratch,
                      COWA_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" cowa_status cowa_decode_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  const cowa_status st = cowa::scratch_on_current_device(&scratch);
+  if (st != COWA_OK) return st;
+  return cowa_workspace_status(scratch, stream);
 }

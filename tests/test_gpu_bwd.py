@@ -99,23 +99,30 @@ def test_bwd_prefill_8k(cuda_device):
 
 
 def test_bwd_train_32k(cuda_device):
-    """B=1, N=T=32768, H_q=40, H_kv=8, d=128, S=128, L=2048, D=8: sampled rows, band-only and
-    late-interval columns, and the any-size identities."""
+    """B=1, N=T=32768, H_q=40, H_kv=8, d=128, S=128, L=2048, D=8: sampled rows; for dk/dv the
+    sink columns and the early-interval columns (the key tiles every later query tile visits:
+    the longest accumulations), every interval edge of KV heads 0 and 1, band-only columns, the
+    late interval of KV head 7 and the last key; and the any-size identities."""
     pat = cw.Pattern(128, 2048, 32768, 8)
     rows = edge_rows(32768, pat, 8, extra_random=96, seed=6)
     band_cols = [5000, 5001, 9000, 20000]
+    sink = [0, 64, 127]
+    head0 = [128, 129, 2000, 4207]        # interval [128, 4208) of KV head 0; 2000 is past the band of row 4100
+    head1 = [4208, 4209, 8287]            # interval [4208, 8288) of KV head 1
     late = [28688, 28700, 30000, 32767]   # interval of KV head 7 and the last key
-    _check_sampled(1, 32768, 40, 8, 128, pat, cuda_device, rows, [(0, band_cols), (7, band_cols + late)],
+    _check_sampled(1, 32768, 40, 8, 128, pat, cuda_device, rows,
+                   [(0, sink + head0 + band_cols), (1, sink[:1] + head1 + [9000]), (7, sink[:1] + band_cols + late)],
                    cuda_gen=True)
 
 
 def test_bwd_long_128k(cuda_device):
-    """B=1, N=T=131072, H_q=40, H_kv=8, d=128, S=128, L=4096, D=8: sampled rows, band-only
-    columns and the any-size identities."""
+    """B=1, N=T=131072, H_q=40, H_kv=8, d=128, S=128, L=4096, D=8: sampled rows; dk/dv at a sink
+    column and the first interval column of KV head 0 (key tiles walked by all 1,024 query
+    tiles), band-only columns, the last key; and the any-size identities."""
     pat = cw.Pattern(128, 4096, 131072, 8)
     rows = np.array([0, 127, 128, 4095, 4096, 16495, 16496, 70000, 131071])
-    _check_sampled(1, 131072, 40, 8, 128, pat, cuda_device, rows, [(3, [20000, 40001]), (7, [131071])],
-                   cuda_gen=True)
+    _check_sampled(1, 131072, 40, 8, 128, pat, cuda_device, rows,
+                   [(0, [5, 128]), (3, [20000, 40001]), (7, [131071])], cuda_gen=True)
 
 
 def test_bwd_stages_on_two_streams_match_single_call(cuda_device):

@@ -1,11 +1,17 @@
 """cowa_decode_noalloc: decode for callers that cannot allocate device memory.
 
-The entry point keeps its split partials in the library's own static per-device scratch
-instead of a caller workspace.  Checked through the C ABI against cowa_decode (which uses a
-caller workspace) on two calls in a row with different inputs, within the decode tolerances
-of the other parity tests; the second call must not see anything left over from the first.
-Also checks that a configuration too large for the scratch is refused before any launch.
-This file is collected last on purpose."""
+Some callers cannot allocate device memory on the serving path (runtimes that own the whole
+memory pool, or code that must not call cudaMalloc because it synchronizes the device).  This
+entry point keeps its split partials in the library's own static per-device scratch instead of
+a caller workspace.  Checked through the C ABI against cowa_decode (which uses a caller
+workspace) on two calls in a row with different inputs, within the decode tolerances of the
+other parity tests; the second call must not see anything left over from the first.  That a
+call allocates nothing is checked twice: torch's allocator count is unchanged, and the device's
+free memory as the driver reports it (cudaMemGetInfo) does not drop across the second call (any
+device allocation, however small, takes at least one 2 MiB page; the first call of a process may
+load the library's device code, whose static scratch is part of that load).  The scratch's status word is read
+back through cowa_decode_noalloc_status.  Also checks that a configuration too large for the
+scratch is refused before any launch.  This file is collected last on purpose."""
 
 import ctypes
 
@@ -42,17 +48,21 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
     ]
     out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=cuda_device)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=cuda_device)
-    for qt, pos_list in calls:
+    for i, (qt, pos_list) in enumerate(calls):
         pos = torch.tensor(pos_list, dtype=torch.int32, device=cuda_device)
         want_o, want_l = cw.cowa_decode(qt, kc, vc, pos, pat)
         torch.cuda.synchronize()
         out.fill_(float("nan"))
         lse.fill_(float("nan"))
         before = torch.cuda.memory_allocated(cuda_device)
+        free_before = torch.cuda.mem_get_info(cuda_device)[0]
         st = _call_noalloc(pat, qt, kc, vc, pos, out, lse)
         torch.cuda.synchronize()
         assert st == 0, cw.lib().cowa_status_string(st)
         assert torch.cuda.memory_allocated(cuda_device) == before
+        if i > 0:  # the first call may load the library's device code, scratch included
+            assert free_before - torch.cuda.mem_get_info(cuda_device)[0] < 2 * 1024 * 1024
+        assert cw.decode_noalloc_status() == 0
         err_o = float((out.float() - want_o.float()).abs().max())
         err_l = float((lse - want_l).abs().max())
         assert np.isfinite(err_o) and np.isfinite(err_l)
