@@ -6,9 +6,11 @@ training layer plus cowa_decode on the 128K decode cache.
 Prints one JSON line (rank 0).  `value` is visible TFLOP/s of the training part
 (forward 4*d and backward 10*d FLOPs per visible query-key pair, summed over all
 ranks) divided by the max-over-ranks device time of the whole step (decode
-included); `parts` gives each call's CUDA-event time, the decode GB/s over the
-visible K/V bytes, and the same for the dense-causal mode when --dense is given;
---sweep adds the other configurations (see `sweep_configs`).
+included); `parts` gives each call's CUDA-event time and the decode GB/s over the
+visible K/V bytes, and also carries the other configurations, each kernel timed alone
+(see `config_parts`): the 32K layer's dense-causal mode and SWA + sinks, the 128K layer
+and its dense-causal mode, and the 128K decode in the dense-causal mode, over the
+compacted cache and over E4M3 caches; --sweep adds the 8K prefill D sweep.
 Inputs are larger than L2 (126 MB), so no flush is needed between steps.
 
 N > 1: one process per GPU (torchrun); every rank runs the same per-GPU workload on
@@ -198,9 +200,16 @@ _KV_CACHE = {}
 
 
 def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
-    """Time the fp64 oracle forward on row blocks of the 32K config until ~target_s of CPU work
-    (input generation is outside the timed part).  Returns (visible TFLOP/s, description,
-    threads, seconds timed)."""
+    """Time the fp64 oracle on random blocks of the 32K layer for about target_s seconds of CPU
+    work (input generation is outside the timed part), half on the forward and half on the
+    backward, and return the whole step's rate at those speeds.
+
+    Forward: attention_fwd_rows on 32-row blocks, 4*d FLOPs credited per visible pair.
+    Backward: attention_bwd_rows on 32-row blocks (the row-local part of the backward: S, dP, dS
+    and dQ), 6*d FLOPs credited per visible pair; that rate stands for the whole 10*d backward
+    (the column-local dK/dV part is the same kind of dense fp64 work).
+    Returns (step TFLOP/s = (fwd + bwd FLOPs of a step) / (the time the oracle would take for
+    them at the two measured rates), fwd TFLOP/s, bwd TFLOP/s, description, threads, seconds)."""
     import numpy as np
 
     from oracle import cowa_oracle as orc
@@ -208,8 +217,9 @@ def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
 
     c = TRAIN
     pat = orc.Pattern(S=c["S"], L=c["L"], T=c["T"], D=c["D"])
-    rng = np.random.default_rng(99)
+    rng = np.random.default_rng(99 + seed_extra)
     Hkv, Hq, d, N = c["Hkv"], c["Hq"], c["d"], c["N"]
+    grp = Hq // Hkv
 
     class Rows:
         """A seeded bf16 tensor widened to float64 on access (the oracle reads slices)."""
@@ -221,68 +231,92 @@ def cpu_oracle_sample(target_s: float, seed_extra: int = 0):
         def __getitem__(self, idx):
             return orc.bf16_bits_to_f64(self.bits[idx])
 
-    if seed_extra not in _KV_CACHE:
+    if seed_extra not in _KV_CACHE:  # generated once per seed, outside the timed parts
         _KV_CACHE[seed_extra] = (Rows("k", Hkv), Rows("v", Hkv))
     k, v = _KV_CACHE[seed_extra]
 
     class QRows:
-        """Query rows drawn per 32-row block (only the sampled rows are ever generated)."""
+        """Query-side rows (q, dO) drawn per accessed block of rows and head: only the sampled
+        rows are ever generated (a few milliseconds per block, against the oracle's ~0.1 s)."""
 
         shape = (1, N, Hq, d)
 
-        def __getitem__(self, idx):
-            b, rows, h, _ = idx
-            rows = np.atleast_1d(rows)
-            blk = synth.normal_bf16_bits((len(rows), d), synth.seed_of("q", seed_extra) + 7919 * int(rows[0]) + h)
-            return orc.bf16_bits_to_f64(blk)
+        def __init__(self, name):
+            self.seed = synth.seed_of(name, seed_extra)
 
-    q = QRows()
-    done_flops, t_used, nblocks = 0.0, 0.0, 0
-    while t_used < target_s and nblocks < 512:
+        def __getitem__(self, idx):
+            _, rows, h, _ = idx
+            rows = np.atleast_1d(rows)
+            return orc.bf16_bits_to_f64(synth.normal_bf16_bits((len(rows), d), self.seed + 7919 * int(rows[0]) + h))
+
+    q, do = QRows("q"), QRows("do")
+
+    def row_pairs(rows):
+        return sum(int(orc.visible_mask(rows, int(rows[-1]) + 1, pat, g, Hkv).sum()) for g in range(Hkv)) * grp
+
+    f_flop = f_t = b_flop = b_t = 0.0
+    nf = nb = 0
+    while (f_t + b_t) < target_s and nf + nb < 1024:
         t0 = int(rng.integers(0, N - 32))
         rows = np.arange(t0, t0 + 32)
         st = time.perf_counter()
-        orc.attention_fwd_rows(q, k, v, pat, rows, b=0)
-        t_used += time.perf_counter() - st
-        pairs = 0
-        for g in range(Hkv):
-            pairs += int(orc.visible_mask(rows, int(rows[-1]) + 1, pat, g, Hkv).sum()) * (Hq // Hkv)
-        done_flops += 4.0 * d * pairs
-        nblocks += 1
+        if f_t <= b_t:
+            orc.attention_fwd_rows(q, k, v, pat, rows, b=0)
+            f_t += time.perf_counter() - st
+            f_flop += 4.0 * d * row_pairs(rows)
+            nf += 1
+        else:
+            orc.attention_bwd_rows(q, k, v, do, pat, rows, b=0)
+            b_t += time.perf_counter() - st
+            b_flop += 6.0 * d * row_pairs(rows)
+            nb += 1
     try:
         from threadpoolctl import threadpool_info
 
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         threads = os.cpu_count() or 1
-    desc = (f"oracle forward (fp64 numpy, explicit mask) on {nblocks} random 32-row blocks x {Hq} heads "
-            f"of the 32K layer, visible FLOPs credited")
-    return done_flops / t_used / 1e12, desc, threads, t_used
+    f_rate, b_rate = f_flop / f_t, b_flop / b_t
+    pairs = visible_pairs(N, c["S"], c["L"], c["T"], c["D"], Hkv, Hq, c["B"])
+    step_flop = 14.0 * d * pairs
+    step_s = 4.0 * d * pairs / f_rate + 10.0 * d * pairs / b_rate
+    desc = (f"oracle (fp64 numpy, explicit mask) on the 32K layer, all {Hq} query heads: forward of {nf} "
+            f"random 32-row blocks (4*d per visible pair) and the row-local backward (S, dP, dS, dQ) of {nb} "
+            f"random 32-row blocks (6*d per pair); value = a step's visible FLOPs (fwd 4*d + bwd 10*d per "
+            f"pair) over the time the oracle takes for them at those two rates")
+    return step_flop / step_s / 1e12, f_rate / 1e12, b_rate / 1e12, desc, threads, f_t + b_t
 
 
-# ------------------------------------------------------------------------------ sweep
-SWEEP = [  # (name, B, N, Hq, Hkv, d, S, L, T, D, bwd)
-    ("prefill 8K D=8", 2, 8192, 32, 8, 128, 128, 1024, 8192, 8, True),
-    ("prefill 8K D=4", 2, 8192, 32, 8, 128, 128, 1024, 8192, 4, False),
-    ("prefill 8K D=2", 2, 8192, 32, 8, 128, 128, 1024, 8192, 2, False),
-    ("prefill 8K D=1", 2, 8192, 32, 8, 128, 128, 1024, 8192, 1, False),
-    ("train 32K dense causal", 1, 32768, 40, 8, 128, 128, 32768, 32768, 8, True),
-    ("train 32K SWA + sinks (T = S)", 1, 32768, 40, 8, 128, 128, 2048, 128, 8, True),
-    ("long 128K", 1, 131072, 40, 8, 128, 128, 4096, 131072, 8, True),
-    ("long 128K dense causal", 1, 131072, 40, 8, 128, 128, 131072, 131072, 8, True),
+# ------------------------------------------------------------------------------ other configurations
+# (key, B, N, Hq, Hkv, d, S, L, T, D, time the backward too, in the default report)
+CONFIGS = [
+    ("train_32k", 1, 32768, 40, 8, 128, 128, 2048, 32768, 8, True, True),
+    ("train_32k_dense_causal", 1, 32768, 40, 8, 128, 128, 32768, 32768, 8, True, True),
+    ("train_32k_swa_sinks", 1, 32768, 40, 8, 128, 128, 2048, 128, 8, True, True),
+    ("long_128k", 1, 131072, 40, 8, 128, 128, 4096, 131072, 8, True, True),
+    ("long_128k_dense_causal", 1, 131072, 40, 8, 128, 128, 131072, 131072, 8, True, True),
+    ("prefill_8k_D8", 2, 8192, 32, 8, 128, 128, 1024, 8192, 8, True, False),
+    ("prefill_8k_D4", 2, 8192, 32, 8, 128, 128, 1024, 8192, 4, False, False),
+    ("prefill_8k_D2", 2, 8192, 32, 8, 128, 128, 1024, 8192, 2, False, False),
+    ("prefill_8k_D1", 2, 8192, 32, 8, 128, 128, 1024, 8192, 1, False, False),
 ]
 
 
-def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
-    """Times cowa_fwd and the three backward stages on each SWEEP configuration and the decode
-    step in the dense-causal mode, CUDA events, median of `reps` after one warm-up.  Fractions
-    are of the measured burst bf16 peak (each kernel runs alone) and of the HBM copy rate."""
+def config_parts(dev, kc, vc, peak_tf, hbm_gbs, sweep=False, reps=2):
+    """Each kernel alone (CUDA events, median of `reps` after one warm-up; fractions of the
+    measured burst bf16 peak and of the HBM copy rate) on the other configurations: the 32K
+    layer itself, its dense-causal mode (L >= T, the FullAttn comparison) and SWA + sinks
+    (T = S), the 128K layer and its dense-causal mode, and the 128K decode over the full
+    cache, in the dense-causal mode, over the compacted cache and over E4M3 caches; `sweep`
+    adds the 8K prefill D sweep.  Returns {key: row}."""
+    import ctypes
+
     import torch
 
     from structured_sparse_attention_cowa_b200 import cowa as cw
     from structured_sparse_attention_cowa_b200 import synth
 
-    out = []
+    out = {}
 
     def timed(fn, inner=1):
         """Median over `reps` of the per-call time of `inner` back-to-back calls between one pair
@@ -291,7 +325,7 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
         fn()
         torch.cuda.synchronize()
         ts = []
-        for _ in range(reps):
+        for _ in range(max(1, reps)):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             for _ in range(inner):
@@ -300,23 +334,25 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
             ts.append(a.elapsed_time(b) / inner)
         return statistics.median(ts)
 
-    for name, B, N, Hq, Hkv, d, S, L, T, D, do_bwd in SWEEP:
+    for key, B, N, Hq, Hkv, d, S, L, T, D, do_bwd, default in CONFIGS:
+        if not (default or sweep):
+            continue
         pat = cw.Pattern(S, L, T, D)
         q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), dev)
         k = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("k"), dev)
         v = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("v"), dev)
         o = torch.empty_like(q)
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        n_ws = cw.lib().cowa_fwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+        ws_f = torch.zeros(max(256, n_ws), dtype=torch.uint8, device=dev)
         pairs = visible_pairs(N, S, L, T, D, Hkv, Hq, B)
-        f_ms = timed(lambda: cw.cowa_fwd(q, k, v, pat, out=o, lse=lse))
-        row = {"config": name, "B": B, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "S": S, "L": L, "T": T, "D": D,
+        f_ms = timed(lambda: cw.cowa_fwd(q, k, v, pat, out=o, lse=lse, workspace=ws_f))
+        row = {"B": B, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "S": S, "L": L, "T": T, "D": D,
                "visible_pairs": pairs, "fwd_ms": f_ms, "fwd_tflops": 4.0 * d * pairs / (f_ms * 1e-3) / 1e12}
         row["fwd_frac_burst"] = row["fwd_tflops"] / peak_tf
         if do_bwd:
             do = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("do"), dev)
             dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-            import ctypes
-
             n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
             ws = torch.zeros(n, dtype=torch.uint8, device=dev)
             stage = lambda st: cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws, stages=st)
@@ -326,59 +362,81 @@ def sweep_configs(dev, kc, vc, peak_tf, hbm_gbs, reps=3):
             row.update({"bwd_ms": b_ms, "bwd_stages_ms": st_ms, "bwd_tflops": 10.0 * d * pairs / (b_ms * 1e-3) / 1e12})
             row["bwd_frac_burst"] = row["bwd_tflops"] / peak_tf
             if cw.workspace_status(ws) != 0:
-                raise RuntimeError(f"device status set in sweep config {name}")
+                raise RuntimeError(f"device status set in configuration {key}")
             del do, dq, dk, dv, ws
-        out.append(row)
-        del q, k, v, o, lse
+        if cw.workspace_status(ws_f) != 0:
+            raise RuntimeError(f"device status set in configuration {key}")
+        out[key] = row
+        del q, k, v, o, lse, ws_f
         torch.cuda.empty_cache()
+    for key in ("train_32k_dense_causal", "long_128k_dense_causal"):
+        base = key.replace("_dense_causal", "")
+        if key in out and base in out:  # CoWA against the dense-causal mode of the same kernels
+            out[key]["cowa_fwd_speedup"] = out[key]["fwd_ms"] / out[base]["fwd_ms"]
+            if "bwd_ms" in out[key] and "bwd_ms" in out[base]:
+                out[key]["cowa_bwd_speedup"] = out[key]["bwd_ms"] / out[base]["bwd_ms"]
 
-    # decode: the CoWA pattern over the full cache, the dense-causal mode (every cached token up
-    # to pos visible) and the CoWA pattern over the compacted cache, timed alike: explicit
-    # workspaces, 10 back-to-back calls per event pair
-    import ctypes
-
+    # decode at 128K (B = 16, pos = 131071): the CoWA pattern over the full cache, the
+    # dense-causal mode (every cached token up to pos visible), the CoWA pattern over the
+    # compacted cache, and over E4M3 caches (full and compacted) quantised from the same values;
+    # all timed alike: explicit workspaces, 10 back-to-back calls per event pair
     dc = DECODE
     L_ = cw.lib()
     qt = synth.cuda_normal_bf16((dc["B"], dc["Hq"], dc["d"]), synth.seed_of("q_t"), dev)
     pos = torch.full((dc["B"],), dc["pos"], dtype=torch.int32, device=dev)
     od = torch.empty((dc["B"], dc["Hq"], dc["d"]), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((dc["B"], dc["Hq"]), dtype=torch.float32, device=dev)
     ws_of = lambda n: torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
     pat_c = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
     toks = decode_visible_tokens(dc["pos"], dc["S"], dc["L"], dc["T"], dc["D"], dc["Hkv"])
     vbytes = float(sum(toks)) * dc["B"] * dc["d"] * 2 * 2
+    shape = (dc["B"], dc["Hq"], dc["Hkv"], dc["d"], dc["T_cap"])
+    wss = []
 
-    ws_c = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(pat_c.c()), dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
-                                                dc["T_cap"]))
-    f_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, pat_c, out=od, workspace=ws_c), inner=10)
-    out.append({"config": "decode 128K (full cache)", "B": dc["B"], "pos": dc["pos"], "decode_ms": f_ms,
-                "decode_gbs": vbytes / (f_ms * 1e-3) / 1e9, "decode_frac_hbm": vbytes / (f_ms * 1e-3) / 1e9 / hbm_gbs,
-                "bytes": vbytes})
+    def dec_row(key, ms, nbytes, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[key] = {"B": dc["B"], "pos": dc["pos"], "decode_ms": ms, "bytes": nbytes, "decode_gbs": gbs,
+                    "decode_frac_hbm": gbs / hbm_gbs, **extra}
+
+    ws_c = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(pat_c.c()), *shape)); wss.append(ws_c)
+    ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, pat_c, out=od, lse=lsed, workspace=ws_c), inner=10)
+    dec_row("decode_128k", ms, vbytes)
+    full_ms = ms
 
     dpat = cw.Pattern(dc["S"], dc["T"], dc["T"], dc["D"])
-    ws_dd = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(dpat.c()), dc["B"], dc["Hq"], dc["Hkv"], dc["d"],
-                                                 dc["T_cap"]))
-    d_ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, dpat, out=od, workspace=ws_dd), inner=10)
-    dbytes = float(dc["pos"] + 1) * dc["B"] * dc["Hkv"] * dc["d"] * 2 * 2
-    out.append({"config": "decode 128K dense causal", "B": dc["B"], "pos": dc["pos"], "decode_ms": d_ms,
-                "decode_gbs": dbytes / (d_ms * 1e-3) / 1e9, "decode_frac_hbm": dbytes / (d_ms * 1e-3) / 1e9 / hbm_gbs,
-                "bytes": dbytes})
+    ws_dd = ws_of(L_.cowa_decode_workspace_size(ctypes.byref(dpat.c()), *shape)); wss.append(ws_dd)
+    ms = timed(lambda: cw.cowa_decode(qt, kc, vc, pos, dpat, out=od, lse=lsed, workspace=ws_dd), inner=10)
+    dec_row("decode_128k_dense_causal", ms, float(dc["pos"] + 1) * dc["B"] * dc["Hkv"] * dc["d"] * 2 * 2,
+            cowa_speedup=ms / full_ms)
 
-    # decode over the compacted per-head cache (sink + band ring + own interval), built from the
-    # full cache; the same visible bytes are read, the cache holds 20,736 instead of 131,072 rows
     kc_c, vc_c = cw.compact_cache(kc.transpose(1, 2), vc.transpose(1, 2), pat_c)
-    ws_k = ws_of(L_.cowa_decode_compact_workspace_size(ctypes.byref(pat_c.c()), dc["B"], dc["Hq"], dc["Hkv"],
-                                                        dc["d"]))
-    c_ms = timed(lambda: cw.cowa_decode_compact(qt, kc_c, vc_c, pos, pat_c, out=od, workspace=ws_k), inner=10)
     rows = cw.compact_rows(pat_c, dc["Hkv"])
-    out.append({"config": "decode 128K over the compacted cache", "B": dc["B"], "pos": dc["pos"], "decode_ms": c_ms,
-                "decode_gbs": vbytes / (c_ms * 1e-3) / 1e9, "decode_frac_hbm": vbytes / (c_ms * 1e-3) / 1e9 / hbm_gbs,
-                "cache_rows_per_head": rows, "full_cache_rows_per_head": dc["T_cap"],
-                "cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * rows * dc["d"] * 2,
-                "full_cache_bytes": 2.0 * dc["B"] * dc["Hkv"] * dc["T_cap"] * dc["d"] * 2})
-    for w in (ws_c, ws_dd, ws_k):
-        if cw.workspace_status(w) != 0:
-            raise RuntimeError("device status set in the decode sweep")
+    ws_k = ws_of(L_.cowa_decode_compact_workspace_size(ctypes.byref(pat_c.c()), *shape[:4])); wss.append(ws_k)
+    ms = timed(lambda: cw.cowa_decode_compact(qt, kc_c, vc_c, pos, pat_c, out=od, lse=lsed, workspace=ws_k),
+               inner=10)
+    cache_full = 2.0 * dc["B"] * dc["Hkv"] * dc["T_cap"] * dc["d"] * 2
+    dec_row("decode_128k_compact", ms, vbytes, cache_rows_per_head=rows, cache_bytes=cache_full * rows / dc["T_cap"],
+            full_cache_bytes=cache_full)
     del kc_c, vc_c
+
+    # E4M3 caches: one scale per tensor (the inputs are N(0,1): |x| < 7 maps below 448 at 1/64)
+    scale = 1.0 / 64
+    kq, vq = cw.quantize_e4m3(kc, scale), cw.quantize_e4m3(vc, scale)
+    ws_8 = ws_of(L_.cowa_decode_fp8_workspace_size(ctypes.byref(pat_c.c()), *shape)); wss.append(ws_8)
+    ms = timed(lambda: cw.cowa_decode_fp8(qt, kq, vq, pos, pat_c, scale, scale, out=od, lse=lsed, workspace=ws_8),
+               inner=10)
+    dec_row("decode_128k_e4m3", ms, vbytes / 2, bf16_decode_ms=full_ms, cache_bytes=cache_full / 2)
+    k8c, v8c = cw.compact_cache_fp8(kq.transpose(1, 2), vq.transpose(1, 2), pat_c)
+    del kq, vq
+    ws_8c = ws_of(L_.cowa_decode_fp8_compact_workspace_size(ctypes.byref(pat_c.c()), *shape[:4])); wss.append(ws_8c)
+    ms = timed(lambda: cw.cowa_decode_fp8_compact(qt, k8c, v8c, pos, pat_c, scale, scale, out=od, lse=lsed,
+                                                  workspace=ws_8c), inner=10)
+    dec_row("decode_128k_e4m3_compact", ms, vbytes / 2, cache_bytes=cache_full * rows / dc["T_cap"] / 2)
+    del k8c, v8c
+    for w in wss:
+        if cw.workspace_status(w) != 0:
+            raise RuntimeError("device status set in the decode configurations")
+    torch.cuda.empty_cache()
     return out
 
 
@@ -560,10 +618,13 @@ def main():
     ap.add_argument("--impl", default="cowa", choices=["cowa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-outputs", default="results", choices=["results", "all"],
-                    help="results: read back the forward lse and the decode output/lse (o, dq, dk, dv stay on "
-                         "the device as in training); all: also copy o, dq, dk, dv out every step")
-    ap.add_argument("--dense", action="store_true", help="also time the dense-causal mode (L >= T)")
+    ap.add_argument("--e2e-outputs", default="all", choices=["results", "all"],
+                    help="all (default): every step copies o, lse, dq, dk, dv and the decode output/lse back to "
+                         "the host, and the line also gives the results-only figure; results: only the forward "
+                         "lse and the decode output/lse (o, dq, dk, dv stay on the device as in training)")
+    ap.add_argument("--no-parts", action="store_true",
+                    help="skip the other configurations (dense-causal mode, SWA + sinks, 128K layer, decode "
+                         "variants) that the line reports under 'parts'")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
                     help="batch: every rank runs the per-GPU workload on its own batch element (weak scaling); "
                          "heads: the one layer split by KV head over the ranks (strong scaling, see run_cowa_tp)")
@@ -571,9 +632,7 @@ def main():
                     help="--shard heads: which global KV heads each rank owns (shard.head_owner)")
     ap.add_argument("--tp-ranks", type=int, default=1,
                     help="--shard heads in one process: run this many ranks' calls in turn on the one GPU")
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time the other configurations (8K prefill D sweep, 128K layer, dense-causal at "
-                         "32K/128K, dense decode) and add them under 'sweep' (one GPU only)")
+    ap.add_argument("--sweep", action="store_true", help="also time the 8K prefill D sweep (one GPU only)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -587,22 +646,26 @@ def main():
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle (test infrastructure) on the host cores, on bounded
+    samples of the same 32K layer (cpu_oracle_sample), one sample per step; rank 0 only."""
     if rank != 0:
         return 0
     steps, warm = max(1, args.steps), max(0, args.warmup)
     per = max(1.0, min(20.0, 120.0 / (steps + warm)))
     vals = []
     for i in range(warm + steps):
-        v, desc, threads, used = cpu_oracle_sample(per, seed_extra=i % 3)
+        v, f_cpu, b_cpu, desc, threads, used = cpu_oracle_sample(per, seed_extra=i % 3)
         if i >= warm:
-            vals.append((v, used))
-    value = statistics.median(v for v, _ in vals)
-    ms = statistics.mean(u for _, u in vals) * 1e3
+            vals.append((v, f_cpu, b_cpu, used))
+    value = statistics.median(x[0] for x in vals)
+    ms = statistics.mean(x[3] for x in vals) * 1e3
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "train 32K layer, oracle forward on row samples", **TRAIN},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "config": {"workload": "train 32K layer fwd+bwd, oracle on row samples", **TRAIN},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+                             "fwd_tflops": statistics.median(x[1] for x in vals),
+                             "bwd_tflops": statistics.median(x[2] for x in vals)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -625,7 +688,6 @@ def run_cowa(args, world, rank, local):
     torch.cuda.set_device(dev)
     c, dc = TRAIN, DECODE
     pat = cw.Pattern(c["S"], c["L"], c["T"], c["D"])
-    pat_dense = cw.Pattern(c["S"], c["N"], c["T"], c["D"])
     dpat = cw.Pattern(dc["S"], dc["L"], dc["T"], dc["D"])
 
     # ---- inputs (per rank: its own batch element / seeds), outputs, workspaces
@@ -724,22 +786,7 @@ def run_cowa(args, world, rank, local):
                    "frac_hbm": dec_bytes / (dec_ms * 1e-3) / 1e9 / hbm, "visible_bytes": dec_bytes},
     }
     for p in ("fwd", "bwd"):
-        parts[p]["frac_peak"] = parts[p]["tflops_visible"] / sustained
-
-    # ---- dense-causal mode (FullAttn comparison), optional
-    if args.dense:
-        def fwd_d():
-            cw.cowa_fwd(q, k, v, pat_dense, out=o, lse=lse, workspace=ws_f)
-        fwd_d(); torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(3):
-            fwd_d()
-        b.record(); torch.cuda.synchronize()
-        dms = a.elapsed_time(b) / 3
-        dpairs = c["N"] * (c["N"] + 1) // 2 * c["Hq"] * c["B"]
-        parts["fwd_dense_causal"] = {"ms": dms, "tflops": 4.0 * c["d"] * dpairs / (dms * 1e-3) / 1e12,
-                                     "speedup_cowa_vs_dense": dms / fwd_ms}
+        parts[p]["frac_peak"] = parts[p]["tflops_visible"] / burst
 
     # ---- roofline of the dominant kernel (longest device time in the step).  Algorithmic work per
     # launch: forward 2 GEMMs (4*d per visible pair), dK/dV 4 GEMMs (S^T, dP^T, dV, dK: 8*d per
@@ -754,9 +801,10 @@ def run_cowa(args, world, rank, local):
     t_ms, work, bound, src, per = kernels[top]
     if bound == "tensor":
         achieved = work / (t_ms * 1e-3) / 1e12
-        roofline = {"kernel": top, "bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                    "frac": achieved / sustained, "traffic": _traffic_record(top, src),
-                    "peak_source": f"{peak_src} bf16 dense, sustained",
+        roofline = {"kernel": top, "bound": "tensor", "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                    "frac": achieved / burst, "frac_of_sustained": achieved / sustained,
+                    "traffic": _traffic_record(top, src),
+                    "peak_source": f"{peak_src} bf16 dense, burst (the timed region is under a second)",
                     "algorithmic": f"{work:.4e} FLOP per launch = {per} x visible pairs ({pairs:.4e})"}
     else:
         achieved = work / (t_ms * 1e-3) / 1e9
@@ -769,10 +817,11 @@ def run_cowa(args, world, rank, local):
     # ---- end to end: host buffers, copies inside the timed region.  Every step copies its inputs
     # (q, k, v, dO of the layer, q_t and pos of the decode; the KV cache is resident device state)
     # in from pinned host memory and reads its results back into pinned host memory: by default
-    # the results a host reads in training and serving -- the forward's lse (the per-row
-    # log-partition a loss is formed from) and the decode output and lse -- while o, dq, dk, dv
-    # stay on the device for the next layer and the optimizer; --e2e-outputs all also copies
-    # o, dq, dk and dv out.  Steps are pipelined the way a training or serving loop prefetches:
+    # every result (o, lse, dq, dk, dv and the decode output and lse); the line also gives the
+    # figure with only the results a host reads in training and serving (the forward's lse, the
+    # per-row log-partition a loss is formed from, and the decode output and lse), o, dq, dk, dv
+    # staying on the device for the next layer and the optimizer.  Steps are pipelined the way a
+    # training or serving loop prefetches:
     # three streams (copy-in, compute, copy-out) and two device buffer sets, so step i+1's
     # inputs land while step i computes and step i's results leave while step i+1 computes.
     # Within a step the forward starts once q, k, v are in (dO lands meanwhile).
@@ -784,102 +833,110 @@ def run_cowa(args, world, rank, local):
         for n, x in zip(names_in, (q, k, v, do, qt)):
             h_in[n].copy_(x)
         h_pos = pos.cpu().pin_memory()
-        all_out = args.e2e_outputs == "all"
-        names_out = ("lse", "od", "lsed") + (("o", "dq", "dk", "dv") if all_out else ())
-        dev_out = {"lse": lse, "od": od, "lsed": lsed, "o": o, "dq": dq, "dk": dk, "dv": dv}
-        h_out = {n: pin(dev_out[n]) for n in names_out}
-        h2d = sum(x.numel() * x.element_size() for x in h_in.values()) + h_pos.numel() * 4
-        d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
-        def buffer_set():
-            st = {n: torch.empty_like(x) for n, x in zip(names_in + ("pos",), (q, k, v, do, qt, pos))}
-            st.update({n: torch.empty_like(x) for n, x in dev_out.items()})
-            st.update({n: torch.zeros_like(x) for n, x in (("ws_f", ws_f), ("ws_b", ws_b), ("ws_d", ws_d))})
-            return st
+        def run_e2e(all_out):
+            names_out = ("lse", "od", "lsed") + (("o", "dq", "dk", "dv") if all_out else ())
+            dev_out = {"lse": lse, "od": od, "lsed": lsed, "o": o, "dq": dq, "dk": dk, "dv": dv}
+            h_out = {n: pin(dev_out[n]) for n in names_out}
+            h2d = sum(x.numel() * x.element_size() for x in h_in.values()) + h_pos.numel() * 4
+            d2h = sum(x.numel() * x.element_size() for x in h_out.values())
 
-        sets = [buffer_set(), buffer_set()]
-        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        inputs_free = [None, None]   # compute of the step that last used the set has read its inputs
-        outputs_free = [None, None]  # copy-out of the step that last used the set is done
-        new_ev = lambda: torch.cuda.Event()
+            def buffer_set():
+                st = {n: torch.empty_like(x) for n, x in zip(names_in + ("pos",), (q, k, v, do, qt, pos))}
+                st.update({n: torch.empty_like(x) for n, x in dev_out.items()})
+                st.update({n: torch.zeros_like(x) for n, x in (("ws_f", ws_f), ("ws_b", ws_b), ("ws_d", ws_d))})
+                return st
 
-        def e2e_step(i):
-            st = sets[i % 2]
-            j = i % 2
-            with torch.cuda.stream(s_in):
-                if inputs_free[j] is not None:
-                    s_in.wait_event(inputs_free[j])
-                for n in ("q", "k", "v"):
-                    st[n].copy_(h_in[n], non_blocking=True)
-                e_qkv = new_ev(); e_qkv.record(s_in)
-                st["do"].copy_(h_in["do"], non_blocking=True)
-                e_do = new_ev(); e_do.record(s_in)
-                st["qt"].copy_(h_in["qt"], non_blocking=True)
-                st["pos"].copy_(h_pos, non_blocking=True)
-                e_dec_in = new_ev(); e_dec_in.record(s_in)
-            with torch.cuda.stream(s_cmp):
-                s_cmp.wait_event(e_qkv)
-                if outputs_free[j] is not None:
-                    s_cmp.wait_event(outputs_free[j])
-                cw.cowa_fwd(st["q"], st["k"], st["v"], pat, out=st["o"], lse=st["lse"], workspace=st["ws_f"])
-                e_fwd = new_ev(); e_fwd.record(s_cmp)
-                s_cmp.wait_event(e_do)
-                cw.cowa_bwd(st["q"], st["k"], st["v"], st["o"], st["lse"], st["do"], pat, dq=st["dq"], dk=st["dk"],
-                            dv=st["dv"], workspace=st["ws_b"])
-                e_bwd = new_ev(); e_bwd.record(s_cmp)
-                s_cmp.wait_event(e_dec_in)
-                cw.cowa_decode(st["qt"], kc, vc, st["pos"], dpat, out=st["od"], lse=st["lsed"], workspace=st["ws_d"])
-                e_cmp = new_ev(); e_cmp.record(s_cmp)
-                inputs_free[j] = e_cmp
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(e_fwd)
-                h_out["lse"].copy_(st["lse"], non_blocking=True)
-                if all_out:
-                    h_out["o"].copy_(st["o"], non_blocking=True)
-                s_out.wait_event(e_bwd)
-                if all_out:
-                    for n in ("dq", "dk", "dv"):
-                        h_out[n].copy_(st[n], non_blocking=True)
-                s_out.wait_event(e_cmp)
-                h_out["od"].copy_(st["od"], non_blocking=True)
-                h_out["lsed"].copy_(st["lsed"], non_blocking=True)
-                e_o = new_ev(); e_o.record(s_out)
-                outputs_free[j] = e_o
+            sets = [buffer_set(), buffer_set()]
+            s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+            inputs_free = [None, None]   # compute of the step that last used the set has read its inputs
+            outputs_free = [None, None]  # copy-out of the step that last used the set is done
+            new_ev = lambda: torch.cuda.Event()
 
-        KE = max(2, K)  # the same number of steps as the device-timed region: pipeline fill amortised alike
-        e2e_step(0); e2e_step(1); torch.cuda.synchronize()
-        barrier()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        main_s = torch.cuda.current_stream(dev)
-        a.record(main_s)
-        for st_ in (s_in, s_cmp, s_out):
-            st_.wait_stream(main_s)
-        for i in range(KE):
-            e2e_step(i)
-        for st_ in (s_in, s_cmp, s_out):
-            main_s.wait_stream(st_)
-        b.record(main_s); torch.cuda.synchronize()
-        barrier()
-        for st_ in sets:
-            for n in ("ws_f", "ws_b", "ws_d"):
-                if cw.workspace_status(st_[n]) != 0:
-                    raise RuntimeError("device status set during the end-to-end steps")
-        e_ms = maxr(a.elapsed_time(b)) / KE
-        e2e = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
-               "pipelined": "copy-in / compute / copy-out streams, two device buffer sets",
-               "outputs_read": list(names_out)}
-        del sets
+            def e2e_step(i):
+                st = sets[i % 2]
+                j = i % 2
+                with torch.cuda.stream(s_in):
+                    if inputs_free[j] is not None:
+                        s_in.wait_event(inputs_free[j])
+                    for n in ("q", "k", "v"):
+                        st[n].copy_(h_in[n], non_blocking=True)
+                    e_qkv = new_ev(); e_qkv.record(s_in)
+                    st["do"].copy_(h_in["do"], non_blocking=True)
+                    e_do = new_ev(); e_do.record(s_in)
+                    st["qt"].copy_(h_in["qt"], non_blocking=True)
+                    st["pos"].copy_(h_pos, non_blocking=True)
+                    e_dec_in = new_ev(); e_dec_in.record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(e_qkv)
+                    if outputs_free[j] is not None:
+                        s_cmp.wait_event(outputs_free[j])
+                    cw.cowa_fwd(st["q"], st["k"], st["v"], pat, out=st["o"], lse=st["lse"], workspace=st["ws_f"])
+                    e_fwd = new_ev(); e_fwd.record(s_cmp)
+                    s_cmp.wait_event(e_do)
+                    cw.cowa_bwd(st["q"], st["k"], st["v"], st["o"], st["lse"], st["do"], pat, dq=st["dq"], dk=st["dk"],
+                                dv=st["dv"], workspace=st["ws_b"])
+                    e_bwd = new_ev(); e_bwd.record(s_cmp)
+                    s_cmp.wait_event(e_dec_in)
+                    cw.cowa_decode(st["qt"], kc, vc, st["pos"], dpat, out=st["od"], lse=st["lsed"], workspace=st["ws_d"])
+                    e_cmp = new_ev(); e_cmp.record(s_cmp)
+                    inputs_free[j] = e_cmp
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(e_fwd)
+                    h_out["lse"].copy_(st["lse"], non_blocking=True)
+                    if all_out:
+                        h_out["o"].copy_(st["o"], non_blocking=True)
+                    s_out.wait_event(e_bwd)
+                    if all_out:
+                        for n in ("dq", "dk", "dv"):
+                            h_out[n].copy_(st[n], non_blocking=True)
+                    s_out.wait_event(e_cmp)
+                    h_out["od"].copy_(st["od"], non_blocking=True)
+                    h_out["lsed"].copy_(st["lsed"], non_blocking=True)
+                    e_o = new_ev(); e_o.record(s_out)
+                    outputs_free[j] = e_o
+
+            KE = max(2, K)  # the same number of steps as the device-timed region: pipeline fill amortised alike
+            e2e_step(0); e2e_step(1); torch.cuda.synchronize()
+            barrier()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            main_s = torch.cuda.current_stream(dev)
+            a.record(main_s)
+            for st_ in (s_in, s_cmp, s_out):
+                st_.wait_stream(main_s)
+            for i in range(KE):
+                e2e_step(i)
+            for st_ in (s_in, s_cmp, s_out):
+                main_s.wait_stream(st_)
+            b.record(main_s); torch.cuda.synchronize()
+            barrier()
+            for st_ in sets:
+                for n in ("ws_f", "ws_b", "ws_d"):
+                    if cw.workspace_status(st_[n]) != 0:
+                        raise RuntimeError("device status set during the end-to-end steps")
+            e_ms = maxr(a.elapsed_time(b)) / KE
+            res = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
+                   "pipelined": "copy-in / compute / copy-out streams, two device buffer sets",
+                   "outputs_read": list(names_out)}
+            del sets
+            return res
+
+        e2e = run_e2e(args.e2e_outputs == "all")
+        if args.e2e_outputs == "all":
+            r = run_e2e(False)
+            e2e["results_only"] = {k_: r[k_] for k_ in ("value", "ms_per_step", "h2d_bytes_per_step",
+                                                         "d2h_bytes_per_step", "outputs_read")}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        v_cpu, desc, threads, _ = cpu_oracle_sample(args.cpu_seconds)
+        v_cpu, f_cpu, b_cpu, desc, threads, _ = cpu_oracle_sample(args.cpu_seconds)
         cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
-               "host_cpus": os.cpu_count()}
+               "fwd_tflops": f_cpu, "bwd_tflops": b_cpu, "host_cpus": os.cpu_count()}
 
-    sweep = None
-    if args.sweep and world == 1:
-        sweep = sweep_configs(dev, kc, vc, burst, hbm)  # each kernel timed alone: burst peak
+    # ---- the other configurations, each kernel timed alone (burst peak), one GPU only
+    if world == 1 and not args.no_parts:
+        parts.update(config_parts(dev, kc, vc, burst, hbm, sweep=args.sweep))
 
     if dist is not None:
         dist.destroy_process_group()
@@ -893,8 +950,6 @@ def run_cowa(args, world, rank, local):
                        "parallelism": f"batch-sharded x{world} (weak)"},
             "parts": parts, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": K * 6, "clocks": clk.summary()}  # fwd 1 + bwd 3 + decode 2 per step
-    if sweep is not None:
-        line["sweep"] = sweep
     print(json.dumps(line), flush=True)
     return 0
 

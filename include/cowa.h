@@ -119,10 +119,11 @@ cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int
  * cu_seqlens[s+1]-1 of q [total, H_q, d], k and v [total, H_kv, d] (cowa_tensor strides; stride_b
  * unused but validated), at positions 0 .. len_s-1 each; o [total, H_q, d]; lse fp32
  * contiguous [H_q, total].  Each sequence gets exactly cowa_fwd over its own rows.
- * cu_seqlens: device int32 [n_seq + 1], non-decreasing from 0 to total (entries outside
- * [0, total] are clamped on the device, so a malformed array cannot make the kernel touch rows
- * outside the tensors).  Workspace: cowa_fwd_varlen_workspace_size (status word + per-sequence
- * tile offsets, computed on the device in the same stream).  Errors as for cowa_fwd. */
+ * cu_seqlens: device int32 [n_seq + 1], non-decreasing from 0 to total (the device clamps the
+ * offsets so that sequences stay in order, disjoint and inside [0, total), so a malformed array
+ * cannot make the kernel touch rows outside the tensors).  Workspace:
+ * cowa_fwd_varlen_workspace_size (status word + a sequence table of tile offsets, first rows
+ * and lengths, computed on the device in the same stream).  Errors as for cowa_fwd. */
 size_t cowa_fwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d);
 cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d,
                             const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
@@ -159,17 +160,19 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int H_q, int 
  * rows cu_seqlens[s] .. cu_seqlens[s+1]-1 of q, o, dO, dq [total, H_q, d] and k, v, dk, dv
  * [total, H_kv, d] (cowa_tensor strides; stride_b unused but validated), each at positions
  * 0 .. len_s-1; lse fp32 contiguous [H_q, total] as cowa_fwd_varlen writes it.  Each sequence gets
- * exactly cowa_bwd over its own rows: the call runs, in stream order and one sequence after
- * another, a strided copy of the sequence's lse rows into the workspace and the three backward
- * kernels on row-offset views (launches grow with n_seq: 3 kernels and 1 copy per non-empty
- * sequence).
- * cu_seqlens: HOST int32 [n_seq + 1], cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seq] =
- * total, every length <= max_len; otherwise COWA_ERR_INVALID_ARG (a length above max_len:
- * COWA_ERR_WORKSPACE) before anything is enqueued.  Workspace:
- * cowa_bwd_varlen_workspace_size(pat, max_len, ...).  Other errors as for cowa_bwd. */
-size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int max_len, int H_q, int H_kv, int d);
-cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, const int32_t* cu_seqlens, int total, int max_len,
-                            int H_q, int H_kv, int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+ * exactly cowa_bwd over its own rows (the pattern is applied the same way in training and
+ * inference, skillfed.io news summary of CoWindow Attention, paragraph 2).  The launches do not
+ * grow with n_seq: one small kernel turns cu_seqlens into a sequence table in the workspace, then
+ * each of the three backward kernels runs once over all sequences (a grid over the bound
+ * total/128 + n_seq of 128-row tiles; every CTA finds its sequence in the table).
+ * cu_seqlens: DEVICE int32 [n_seq + 1], non-decreasing from 0 to total.  The device clamps the
+ * offsets so that sequences stay in order, disjoint and inside [0, total) (a malformed table
+ * cannot reach memory outside the tensors; its sequences are then the clamped ones).
+ * Workspace: cowa_bwd_varlen_workspace_size(pat, n_seq, total, ...).  Other errors as for
+ * cowa_bwd. */
+size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d);
+cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d,
+                            const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
                             const float* lse, cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
                             void* ws, size_t ws_bytes, void* stream);
 

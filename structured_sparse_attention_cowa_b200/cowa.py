@@ -99,9 +99,9 @@ def lib() -> ctypes.CDLL:
     L.cowa_bwd.restype = i
     L.cowa_bwd_stages.argtypes = [P, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, i, vp, sz, vp]
     L.cowa_bwd_stages.restype = i
-    L.cowa_bwd_varlen_workspace_size.argtypes = [P, i, i, i, i]
+    L.cowa_bwd_varlen_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_bwd_varlen_workspace_size.restype = sz
-    L.cowa_bwd_varlen.argtypes = [P, i, vp, i, i, i, i, i, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
+    L.cowa_bwd_varlen.argtypes = [P, i, i, i, i, i, vp, T, T, T, T, vp, T, T, T, T, vp, sz, vp]
     L.cowa_bwd_varlen.restype = i
     L.cowa_decode_workspace_size.argtypes = [P, i, i, i, i, i]
     L.cowa_decode_workspace_size.restype = sz
@@ -305,34 +305,29 @@ def cowa_bwd(q, k, v, o, lse, do, pattern: Pattern, dq=None, dk=None, dv=None, w
 def cowa_bwd_varlen(q, k, v, o, lse, do, cu_seqlens, pattern: Pattern, dq=None, dk=None, dv=None, workspace=None,
                     stream=None):
     """Gradients of cowa_fwd_varlen: q, o, do [total, H_q, d], k, v [total, H_kv, d], lse [H_q, total],
-    cu_seqlens on the HOST (list, numpy array or CPU tensor of n_seq + 1 offsets); returns dq, dk, dv.
-    One sequence after another in stream order (see cowa_bwd_varlen in cowa.h)."""
+    cu_seqlens a CUDA int32 tensor of n_seq + 1 offsets (as for cowa_fwd_varlen); returns dq, dk, dv.
+    One launch per backward kernel over all sequences (see cowa_bwd_varlen in cowa.h)."""
     import torch
 
     for n_, x_ in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
         _bf16_cuda(n_, x_)
-    cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
-                                         dtype=np.int64))
-    if cu.ndim != 1 or cu.size < 2 or cu.min() < 0 or cu.max() > 2**31 - 1:
-        raise ValueError("cu_seqlens must be a 1-D host array of n_seq + 1 offsets")
-    cu = cu.astype(np.int32)
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D CUDA int32 tensor")
     total, Hq, d = q.shape
     Hkv = k.shape[1]
-    n_seq = cu.size - 1
-    max_len = max(1, int(np.diff(cu).max()))
+    n_seq = cu_seqlens.numel() - 1
     dq = torch.empty_like(q, memory_format=torch.contiguous_format) if dq is None else dq
     dk = torch.empty_like(k, memory_format=torch.contiguous_format) if dk is None else dk
     dv = torch.empty_like(v, memory_format=torch.contiguous_format) if dv is None else dv
     pat = pattern.c()
     L = lib()
-    ws_bytes = L.cowa_bwd_varlen_workspace_size(ctypes.byref(pat), max_len, Hq, Hkv, d)
+    ws_bytes = L.cowa_bwd_varlen_workspace_size(ctypes.byref(pat), n_seq, total, Hq, Hkv, d)
     if workspace is None:
         workspace = _workspace(ws_bytes, q.device)
     t4 = lambda x: _t4(x.unsqueeze(0))
-    _check("cowa_bwd_varlen", L.cowa_bwd_varlen(ctypes.byref(pat), n_seq, cu.ctypes.data_as(ctypes.c_void_p), total,
-                                                max_len, Hq, Hkv, d, t4(q), t4(k), t4(v), t4(o), lse.data_ptr(),
-                                                t4(do), t4(dq), t4(dk), t4(dv), workspace.data_ptr(),
-                                                workspace.numel(), _stream(stream)))
+    _check("cowa_bwd_varlen", L.cowa_bwd_varlen(ctypes.byref(pat), n_seq, total, Hq, Hkv, d, cu_seqlens.data_ptr(),
+                                                t4(q), t4(k), t4(v), t4(o), lse.data_ptr(), t4(do), t4(dq), t4(dk),
+                                                t4(dv), workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return dq, dk, dv
 
 

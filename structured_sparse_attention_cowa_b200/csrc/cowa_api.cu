@@ -450,7 +450,7 @@ cowa_status cowa_fwd_chunk(const cowa_pattern* pat, int B, int N_q, int N_k, int
 size_t cowa_fwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d) {
   Pat p;
   if (n_seq < 1 || check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, total, Hq, Hkv, d) != COWA_OK) return 0;
-  return kWsHeader + fwd_varlen_workspace_bytes(n_seq);
+  return kWsHeader + seq_table_bytes(n_seq);
 }
 
 cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d,
@@ -472,7 +472,7 @@ cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H
   a.pat = p; a.B = 1; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
   a.Nq = total; a.Nk = total; a.q_off = 0;
   a.varlen = 1; a.n_seq = n_seq; a.total = total; a.cu_seqlens = cu_seqlens;
-  a.tile_off = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.seq_tab = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + kWsHeader);
   a.o = o.ptr; a.o_sb = 0; a.o_st = o.stride_t; a.o_sh = o.stride_h;
   a.lse = lse;
   a.status = reinterpret_cast<uint32_t*>(ws);
@@ -522,6 +522,7 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int H
   a.dk = dk.ptr; a.dk_sb = dk.stride_b; a.dk_st = dk.stride_t; a.dk_sh = dk.stride_h;
   a.dv = dv.ptr; a.dv_sb = dv.stride_b; a.dv_st = dv.stride_t; a.dv_sh = dv.stride_h;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.lse_ld = N;
   a.N_pad = (N + 127) / 128 * 128;
   a.delta = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
   a.lse2 = a.delta + (size_t)B * Hq * a.N_pad;
@@ -537,58 +538,61 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int H
 
 // ------------------------------------------------------------------------------ packed backward
 namespace {
-// workspace of the packed backward: [header + backward statistics for max_len rows][lse scratch]
-size_t bwd_varlen_stats_bytes(int max_len, int Hq, int Hkv, int d) {
-  return kWsHeader + bwd_workspace_bytes(1, max_len, Hq, Hkv, d);
-}
-cowa_tensor rows_from(const cowa_tensor& t, int row0) {
-  cowa_tensor r = t;
-  r.ptr = static_cast<char*>(t.ptr) + (int64_t)row0 * t.stride_t * 2;
-  return r;
-}
+// 128 x the tile bound of a packed batch: every sequence's statistics start at its own tile
+long long packed_rows_pad(int total, int n_seq) { return packed_tiles_bound(total, n_seq) * 128; }
 }  // namespace
 
-size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int max_len, int Hq, int Hkv, int d) {
+size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d) {
   Pat p;
-  if (check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, max_len, Hq, Hkv, d) != COWA_OK) return 0;
-  return bwd_varlen_stats_bytes(max_len, Hq, Hkv, d) + align_up((size_t)Hq * max_len * sizeof(float), 256);
+  if (n_seq < 1 || check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, total, Hq, Hkv, d) != COWA_OK) return 0;
+  const long long rows = packed_rows_pad(total, n_seq);
+  if (rows > 0x7fffffffLL) return 0;
+  return kWsHeader + seq_table_bytes(n_seq) + align_up(2 * (size_t)Hq * (size_t)rows * sizeof(float), 256);
 }
 
-cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, const int32_t* cu_seqlens, int total, int max_len,
-                            int Hq, int Hkv, int d, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
+cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d,
+                            const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
                             const float* lse, cowa_tensor dO, cowa_tensor dq, cowa_tensor dk, cowa_tensor dv,
                             void* ws, size_t ws_bytes, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
   COWA_TRY(check_heads(1, total, Hq, Hkv, d));
-  COWA_TRY(check_heads(1, max_len, Hq, Hkv, d));
   if (n_seq < 1 || !cu_seqlens || !lse) return COWA_ERR_INVALID_ARG;
-  if (cu_seqlens[0] != 0 || cu_seqlens[n_seq] != total) return COWA_ERR_INVALID_ARG;
-  for (int s = 0; s < n_seq; ++s) {
-    if (cu_seqlens[s + 1] < cu_seqlens[s]) return COWA_ERR_INVALID_ARG;
-    if (cu_seqlens[s + 1] - cu_seqlens[s] > max_len) return COWA_ERR_WORKSPACE;
-  }
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return COWA_ERR_ALIGNMENT;
   const cowa_tensor* all[] = {&q, &k, &v, &o, &dO, &dq, &dk, &dv};
   for (const cowa_tensor* t : all) COWA_TRY(check_tensor(*t));
-  if (reinterpret_cast<uintptr_t>(lse) & 3u) return COWA_ERR_ALIGNMENT;
-  COWA_TRY(check_ws(ws, ws_bytes, cowa_bwd_varlen_workspace_size(pat, max_len, Hq, Hkv, d)));
+  const size_t need = cowa_bwd_varlen_workspace_size(pat, n_seq, total, Hq, Hkv, d);
+  if (need == 0) return COWA_ERR_INVALID_ARG;
+  COWA_TRY(check_ws(ws, ws_bytes, need));
 
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.pat = p; a.B = 1; a.N = total; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+  a.varlen = 1; a.n_seq = n_seq; a.total = total;
+  a.seq_tab = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + kWsHeader);
+  a.o = o.ptr; a.o_sb = 0; a.o_st = o.stride_t; a.o_sh = o.stride_h;
+  a.dO = dO.ptr; a.do_sb = 0; a.do_st = dO.stride_t; a.do_sh = dO.stride_h;
+  a.lse = lse;
+  a.lse_ld = total;
+  a.dq = dq.ptr; a.dq_sb = 0; a.dq_st = dq.stride_t; a.dq_sh = dq.stride_h;
+  a.dk = dk.ptr; a.dk_sb = 0; a.dk_st = dk.stride_t; a.dk_sh = dk.stride_h;
+  a.dv = dv.ptr; a.dv_sb = 0; a.dv_st = dv.stride_t; a.dv_sh = dv.stride_h;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.N_pad = (int)packed_rows_pad(total, n_seq);
+  a.delta = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader + seq_table_bytes(n_seq));
+  a.lse2 = a.delta + (size_t)Hq * a.N_pad;
+  a.scale = scale_of(pat, d);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  if (!make_tmap_bf16(&a.tm_q, q.ptr, d, total, Hq, 1, q.stride_t, q.stride_h, q.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_k, k.ptr, d, total, Hkv, 1, k.stride_t, k.stride_h, k.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_v, v.ptr, d, total, Hkv, 1, v.stride_t, v.stride_h, v.stride_b, 128) ||
+      !make_tmap_bf16(&a.tm_do, dO.ptr, d, total, Hq, 1, dO.stride_t, dO.stride_h, dO.stride_b, 128))
+    return COWA_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t stats = bwd_varlen_stats_bytes(max_len, Hq, Hkv, d);
-  float* lse_seq = reinterpret_cast<float*>(static_cast<char*>(ws) + stats);
-  for (int s = 0; s < n_seq; ++s) {
-    const int row0 = cu_seqlens[s], len = cu_seqlens[s + 1] - row0;
-    if (len == 0) continue;
-    // the sequence's lse rows: H_q rows of len floats, pitch total -> contiguous [H_q, len]
-    if (cudaMemcpy2DAsync(lse_seq, (size_t)len * sizeof(float), lse + row0, (size_t)total * sizeof(float),
-                          (size_t)len * sizeof(float), (size_t)Hq, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
-      return COWA_ERR_CUDA;
-    COWA_TRY(cowa_bwd_stages(pat, 1, len, Hq, Hkv, d, rows_from(q, row0), rows_from(k, row0), rows_from(v, row0),
-                             rows_from(o, row0), lse_seq, rows_from(dO, row0), rows_from(dq, row0),
-                             rows_from(dk, row0), rows_from(dv, row0),
-                             COWA_BWD_PREPROCESS | COWA_BWD_DKDV | COWA_BWD_DQ, ws, stats, stream));
-  }
-  return COWA_OK;
+  if (launch_seq_table(cu_seqlens, n_seq, total, a.seq_tab, st) != cudaSuccess) return COWA_ERR_CUDA;
+  return launch_bwd(a, COWA_BWD_PREPROCESS | COWA_BWD_DKDV | COWA_BWD_DQ, st) == cudaSuccess ? COWA_OK
+                                                                                            : COWA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------------------ introspection

@@ -72,17 +72,28 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int LPR = D / 8;            // lanes per row
   constexpr int RPI = 256 / LPR;        // rows per iteration of the block
-  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // tile tg of the statistics: tile i of batch b, or of the sequence it falls in (packed batch)
+  int i = tg, row0 = 0, N = a.N;
+  if (a.varlen) {
+    if (tg >= a.seq_tab[a.n_seq]) return;  // past the last sequence: no statistics read there
+    const int sq = seq_of_tile(a.seq_tab, a.n_seq, tg);
+    i = tg - a.seq_tab[sq];
+    row0 = a.seq_tab[a.n_seq + 1 + sq];
+    N = a.seq_tab[2 * a.n_seq + 1 + sq];
+  }
   const int sub = threadIdx.x % LPR, rr = threadIdx.x / LPR;
-  const size_t base = ((size_t)b * a.Hq + h) * a.N_pad;
+  const size_t base = ((size_t)b * a.Hq + h) * a.N_pad + (size_t)tg * kTile;
+  const size_t lse_base = ((size_t)b * a.Hq + h) * a.lse_ld + row0;
   for (int r = rr; r < kTile; r += RPI) {
-    const int t = i * kTile + r;
+    const int t = i * kTile + r;  // row within the sequence
     float acc = 0.f;
-    if (t < a.N) {
+    if (t < N) {
+      const int64_t row = (int64_t)row0 + t;
       const uint4 ov = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.o) + b * a.o_sb +
-                                                      (int64_t)t * a.o_st + h * a.o_sh + sub * 8);
+                                                      row * a.o_st + h * a.o_sh + sub * 8);
       const uint4 dv = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(a.dO) + b * a.do_sb +
-                                                      (int64_t)t * a.do_st + h * a.do_sh + sub * 8);
+                                                      row * a.do_st + h * a.do_sh + sub * 8);
       const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -93,8 +104,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __grid_consta
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (sub == 0) {
-      a.delta[base + t] = acc;
-      a.lse2[base + t] = t < a.N ? a.lse[((size_t)b * a.Hq + h) * a.N + t] * 1.4426950408889634f : INFINITY;
+      a.delta[base + r] = acc;
+      a.lse2[base + r] = t < N ? a.lse[lse_base + t] * 1.4426950408889634f : INFINITY;
     }
   }
 }
@@ -127,12 +138,22 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = a.Hq / a.Hkv;
   // lowest key tiles first: their query ranges (sink, early intervals) are the longest
-  const int j = blockIdx.x / (a.Hkv * a.B);
+  int j = blockIdx.x / (a.Hkv * a.B);
   const int rem = blockIdx.x % (a.Hkv * a.B);
   const int g = rem % a.Hkv, b = rem / a.Hkv;
-  const int s0 = j * kTile, s1 = imin(a.N, s0 + kTile);
+  // the rows of this CTA's sequence: [row0, row0 + N) of the token axis; statistics tiles from tile0
+  int row0 = 0, N = a.N, tile0 = 0;
+  if (a.varlen) {
+    if (j >= a.seq_tab[a.n_seq]) return;  // whole CTA, before any barrier or TMEM use
+    const int sq = seq_of_tile(a.seq_tab, a.n_seq, j);
+    tile0 = a.seq_tab[sq];
+    j -= tile0;
+    row0 = a.seq_tab[a.n_seq + 1 + sq];
+    N = a.seq_tab[2 * a.n_seq + 1 + sq];
+  }
+  const int s0 = j * kTile, s1 = imin(N, s0 + kTile);
   const Range iv = interval_of(a.pat, g);
-  const Range rows = bwd_row_range(a.pat, iv, s0, s1, a.N);
+  const Range rows = bwd_row_range(a.pat, iv, s0, s1, N);
   const int i_lo = rows.lo / kTile, i_hi = (rows.hi + kTile - 1) / kTile;
   const int nsteps = (i_hi - i_lo) * grp;
 
@@ -168,8 +189,8 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
       ptx::tma_prefetch_desc(&a.tm_do);
       ptx::mbar_arrive_expect_tx(&kv_full, 2 * Geo::kTileBytes);
       for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sK + u * 16384, &a.tm_k, &kv_full, u * 64, s0, g, b);
-        ptx::tma_load_4d(sV + u * 16384, &a.tm_v, &kv_full, u * 64, s0, g, b);
+        ptx::tma_load_4d(sK + u * 16384, &a.tm_k, &kv_full, u * 64, row0 + s0, g, b);
+        ptx::tma_load_4d(sV + u * 16384, &a.tm_v, &kv_full, u * 64, row0 + s0, g, b);
       }
       int issued = 0;
       for (int n = 0; n < nsteps; ++n) {
@@ -179,10 +200,11 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
         uint8_t* dst = sSlot + slot * Geo::kSlotKV;
         ptx::mbar_arrive_expect_tx(&slot_full[slot], Geo::kSlotKV);
         for (int u = 0; u < D / 64; ++u) {
-          ptx::tma_load_4d(dst + u * 16384, &a.tm_q, &slot_full[slot], u * 64, i * kTile, h, b);
-          ptx::tma_load_4d(dst + Geo::kTileBytes + u * 16384, &a.tm_do, &slot_full[slot], u * 64, i * kTile, h, b);
+          ptx::tma_load_4d(dst + u * 16384, &a.tm_q, &slot_full[slot], u * 64, row0 + i * kTile, h, b);
+          ptx::tma_load_4d(dst + Geo::kTileBytes + u * 16384, &a.tm_do, &slot_full[slot], u * 64, row0 + i * kTile,
+                           h, b);
         }
-        const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + (size_t)i * kTile;
+        const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + (size_t)(tile0 + i) * kTile;
         ptx::bulk_load(dst + 2 * Geo::kTileBytes, a.lse2 + so, 512, &slot_full[slot]);
         ptx::bulk_load(dst + 2 * Geo::kTileBytes + 512, a.delta + so, 512, &slot_full[slot]);
         issued = n + 1;
@@ -254,7 +276,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
     const int s = s0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const bool special = s < a.pat.S || (s >= iv.lo && s < iv.hi);
-    const int t_hi = special ? a.N : imin(a.N, s + a.pat.L);  // rows [s, t_hi) see key s
+    const int t_hi = special ? N : imin(N, s + a.pat.L);  // rows [s, t_hi) see key s
     const float sl2 = a.scale_log2;
     bool ok = true;
     // query tile of the current step and its two sub-steps' mask flags, advanced incrementally
@@ -263,7 +285,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
     auto masks_of = [&](int i, bool* nm) {
       for (int x = 0; x < 2; ++x) {
         const int u0 = i * kTile + x * kSub;
-        nm[x] = !tile_full(a.pat, iv, u0, imin(a.N, u0 + kSub), s0, s1);
+        nm[x] = !tile_full(a.pat, iv, u0, imin(N, u0 + kSub), s0, s1);
       }
     };
     bool nm[2];
@@ -291,7 +313,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
       ptx::tmem_wait_ld();
       const float* stat = reinterpret_cast<const float*>(sSlot + (n & 1) * Geo::kSlotKV + 2 * Geo::kTileBytes) +
                           hq * kSub + CW * part;
-      const bool use_poly = !need_mask && t0 + kSub <= a.N;
+      const bool use_poly = !need_mask && t0 + kSub <= N;
       // the element loop is instantiated with and without the mask, chosen once per sub-step
       auto body = [&](auto masked) {
         constexpr bool kMask = decltype(masked)::value;
@@ -347,10 +369,10 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
         ptx::tmem_ld32(lane_base + Geo::kColAcc + D + part * HC + c * 32, dkv + c * 32);
       }
       ptx::tmem_wait_ld();
-      if (s < a.N) {
-        __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + (int64_t)s * a.dv_st +
+      if (s < N) {
+        __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + ((int64_t)row0 + s) * a.dv_st +
                              g * a.dv_sh + part * HC;
-        __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + (int64_t)s * a.dk_st +
+        __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + ((int64_t)row0 + s) * a.dk_st +
                              g * a.dk_sh + part * HC;
 #pragma unroll
         for (int c8 = 0; c8 < HC / 8; ++c8) {
@@ -398,13 +420,25 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = a.Hq / a.Hkv;
-  const int nq = (a.N + kTile - 1) / kTile;
   const int per_i = a.B * a.Hq;
-  const int i = nq - 1 - (int)(blockIdx.x / per_i);  // heaviest (last) query tiles first
+  // heaviest (last) query tiles first; the rows of this CTA's sequence are [row0, row0 + N) of
+  // the token axis, its statistics tiles start at tile0
+  int i, row0 = 0, N = a.N, tile0 = 0;
+  if (!a.varlen) {
+    i = (a.N + kTile - 1) / kTile - 1 - (int)(blockIdx.x / per_i);
+  } else {
+    const int tg = a.seq_tab[a.n_seq] - 1 - (int)(blockIdx.x / per_i);
+    if (tg < 0) return;  // whole CTA, before any barrier or TMEM use
+    const int sq = seq_of_tile(a.seq_tab, a.n_seq, tg);
+    tile0 = a.seq_tab[sq];
+    i = tg - tile0;
+    row0 = a.seq_tab[a.n_seq + 1 + sq];
+    N = a.seq_tab[2 * a.n_seq + 1 + sq];
+  }
   const int rem = blockIdx.x % per_i;
   const int h = rem % a.Hq, b = rem / a.Hq;
   const int g = h / grp;
-  const int t0 = i * kTile, t1 = imin(a.N, t0 + kTile);
+  const int t0 = i * kTile, t1 = imin(N, t0 + kTile);
   const Range iv = interval_of(a.pat, g);
   const Tiles T = plan_tiles(a.pat, iv, t0, t1);
   const int ntiles = T.count;
@@ -444,8 +478,8 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
       ptx::tma_prefetch_desc(&a.tm_v);
       ptx::mbar_arrive_expect_tx(&q_full, 2 * Geo::kTileBytes);
       for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, t0, h, b);
-        ptx::tma_load_4d(sDO + u * 16384, &a.tm_do, &q_full, u * 64, t0, h, b);
+        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + t0, h, b);
+        ptx::tma_load_4d(sDO + u * 16384, &a.tm_do, &q_full, u * 64, row0 + t0, h, b);
       }
       TileCursor cur;
       cur.init(T);
@@ -455,14 +489,16 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
         if (n >= KS && !ptx::mbar_wait(&k_empty[ks], ((n / KS) - 1) & 1, &abort_flag, a.status)) break;
         ptx::mbar_arrive_expect_tx(&k_full[ks], Geo::kTileBytes);
         for (int u = 0; u < D / 64; ++u)
-          ptx::tma_load_4d(sK + ks * Geo::kTileBytes + u * 16384, &a.tm_k, &k_full[ks], u * 64, cur.j * kTile, g, b);
+          ptx::tma_load_4d(sK + ks * Geo::kTileBytes + u * 16384, &a.tm_k, &k_full[ks], u * 64, row0 + cur.j * kTile,
+                           g, b);
         if (n >= VS && !ptx::mbar_wait(&v_empty[vs], ((n / VS) - 1) & 1, &abort_flag, a.status)) {
           issued = -(n + 1);  // K of tile n is in flight, V is not
           break;
         }
         ptx::mbar_arrive_expect_tx(&v_full[vs], Geo::kTileBytes);
         for (int u = 0; u < D / 64; ++u)
-          ptx::tma_load_4d(sV + vs * Geo::kTileBytes + u * 16384, &a.tm_v, &v_full[vs], u * 64, cur.j * kTile, g, b);
+          ptx::tma_load_4d(sV + vs * Geo::kTileBytes + u * 16384, &a.tm_v, &v_full[vs], u * 64, row0 + cur.j * kTile,
+                           g, b);
         issued = n + 1;
       }
       // drain: every copy issued must have landed before the CTA exits
@@ -530,7 +566,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
     const int r = quad * 32 + lane;  // query row = TMEM lane
     const int t = t0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + t;
+    const size_t so = ((size_t)b * a.Hq + h) * a.N_pad + (size_t)(tile0 + i) * kTile + r;
     const float lse2 = a.lse2[so], delta = a.delta[so];
     const float sl2 = a.scale_log2;
     // visible key ranges of row t (absolute positions)
@@ -542,7 +578,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
     cur.init(T);
     for (int n = 0; n < ntiles; ++n, cur.next(T)) {
       const int s0 = cur.j * kTile;
-      const bool need_mask = (s0 + kTile > a.N) || !tile_full(a.pat, iv, t0, t1, s0, imin(a.N, s0 + kTile));
+      const bool need_mask = (s0 + kTile > N) || !tile_full(a.pat, iv, t0, t1, s0, imin(N, s0 + kTile));
       if (!(ok = ptx::mbar_wait_warp(&sdp_full, n & 1, &abort_flag, a.status))) break;
       ptx::tc_fence_after();
       uint32_t sv[CW], pv[CW];
@@ -559,7 +595,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&consumed_dp);  // dP columns too
-      const bool use_poly = !need_mask && t < a.N;
+      const bool use_poly = !need_mask && t < N;
       // dS buffer n & 1 was last read by dQ(n-2), which the commit of S(n) covers.  The element
       // loop is instantiated with and without the mask, chosen once per tile.
       auto chunks = [&](auto masked) {
@@ -602,8 +638,8 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
 #pragma unroll
       for (int c = 0; c < HC / 32; ++c) ptx::tmem_ld32(lane_base + Geo::kColAcc + part * HC + c * 32, dqv + c * 32);
       ptx::tmem_wait_ld();
-      if (t < a.N) {
-        __nv_bfloat16* dqr = reinterpret_cast<__nv_bfloat16*>(a.dq) + b * a.dq_sb + (int64_t)t * a.dq_st +
+      if (t < N) {
+        __nv_bfloat16* dqr = reinterpret_cast<__nv_bfloat16*>(a.dq) + b * a.dq_sb + ((int64_t)row0 + t) * a.dq_st +
                              h * a.dq_sh + part * HC;
 #pragma unroll
         for (int c8 = 0; c8 < HC / 8; ++c8) {

@@ -97,19 +97,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
     i = (a.Nq + kBM - 1) / kBM - 1 - (int)(blockIdx.x / per_i);
   } else {
     // the grid is an upper bound on the q-tiles of the packed batch: find this CTA's sequence
-    const int tiles = a.tile_off[a.n_seq];
+    const int tiles = a.seq_tab[a.n_seq];
     const int tg = tiles - 1 - (int)(blockIdx.x / per_i);
     if (tg < 0) return;  // whole CTA, before any barrier or TMEM use
-    int lo = 0, hi = a.n_seq - 1;  // largest s with tile_off[s] <= tg
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (a.tile_off[mid] <= tg) lo = mid; else hi = mid - 1;
-    }
-    i = tg - a.tile_off[lo];
-    const int st = imin(imax(a.cu_seqlens[lo], 0), a.total);
-    const int en = imin(imax(a.cu_seqlens[lo + 1], st), a.total);
-    row0 = st;
-    Nq = Nk = en - st;
+    const int sq = seq_of_tile(a.seq_tab, a.n_seq, tg);
+    i = tg - a.seq_tab[sq];
+    row0 = a.seq_tab[a.n_seq + 1 + sq];
+    Nq = Nk = a.seq_tab[2 * a.n_seq + 1 + sq];
     q_off = 0;
   }
   int rem = blockIdx.x % per_i;
@@ -516,18 +510,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
   }
 }
 
-// tile_off[s] = q-tiles of the sequences before s (lengths clamped into [0, total]); one thread:
-// the scan is over the handful of sequences of one batch
-__global__ void varlen_tiles_kernel(const int32_t* cu, int n_seq, int total, int32_t* tile_off) {
+// The sequence table of a packed batch (kernel_common.cuh) from cu_seqlens; one thread: the
+// scan is over the sequences of one batch
+__global__ void seq_table_kernel(const int32_t* cu, int n_seq, int total, int32_t* tab) {
   if (threadIdx.x != 0) return;
-  int off = 0;
+  int off = 0, prev_end = 0;
   for (int s = 0; s < n_seq; ++s) {
-    tile_off[s] = off;
-    const int st = imin(imax(cu[s], 0), total);
+    const int st = imin(imax(cu[s], prev_end), total);
     const int en = imin(imax(cu[s + 1], st), total);
+    tab[s] = off;
+    tab[n_seq + 1 + s] = st;
+    tab[2 * n_seq + 1 + s] = en - st;
     off += (en - st + kBM - 1) / kBM;
+    prev_end = en;
   }
-  tile_off[n_seq] = off;
+  tab[n_seq] = off;
 }
 
 template <int D>
@@ -538,8 +535,8 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grp = a.Hq / a.Hkv;
   // packed batch: an upper bound on the q-tiles (sum of ceil(len/BM) <= total/BM + n_seq); the
-  // tile offsets are computed on the device first
-  const long long nq = a.varlen ? (long long)a.total / kBM + a.n_seq : (a.Nq + kBM - 1) / kBM;
+  // sequence table is computed on the device first
+  const long long nq = a.varlen ? packed_tiles_bound(a.total, a.n_seq) : (a.Nq + kBM - 1) / kBM;
   const long long nblk = nq * a.B * a.Hkv * ((grp + 1) / 2);
   if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
   // the in-kernel register split assumes the compiled count equals the launch allocation
@@ -551,8 +548,7 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
   if (a.varlen) {
-    varlen_tiles_kernel<<<1, 32, 0, s>>>(a.cu_seqlens, a.n_seq, a.total, a.tile_off);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_seq_table(a.cu_seqlens, a.n_seq, a.total, a.seq_tab, s)) != cudaSuccess) return e;
   }
   kern<<<(unsigned)nblk, kFwdThreads, Geo::kSmem, s>>>(a);
   return cudaGetLastError();
@@ -560,7 +556,10 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-size_t fwd_varlen_workspace_bytes(int n_seq) { return ((size_t)(n_seq + 1) * sizeof(int32_t) + 255) / 256 * 256; }
+cudaError_t launch_seq_table(const int32_t* cu_seqlens, int n_seq, int total, int32_t* tab, cudaStream_t s) {
+  seq_table_kernel<<<1, 32, 0, s>>>(cu_seqlens, n_seq, total, tab);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s) {
   if (a.d == 64) return launch_fwd_d<64>(a, s);

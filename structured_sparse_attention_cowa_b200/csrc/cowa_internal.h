@@ -71,10 +71,11 @@ struct FwdArgs {
   int B, Hq, Hkv, d;
   int Nq, Nk, q_off;  // query rows q_off .. q_off+Nq-1 (absolute positions) against keys 0 .. Nk-1
   // packed variable-length batch (varlen != 0): sequence s holds rows cu_seqlens[s] ..
-  // cu_seqlens[s+1]-1 of q, k, v, o (B = 1) at positions 0..; tile_off[s] = q-tiles before it
+  // cu_seqlens[s+1]-1 of q, k, v, o (B = 1) at positions 0..; seq_tab is the sequence table
+  // of kernel_common.cuh (tile offsets, first rows, lengths), written first on the device
   int varlen, n_seq, total;
   const int32_t* cu_seqlens;
-  int32_t* tile_off;
+  int32_t* seq_tab;
   void* o;
   int64_t o_sb, o_st, o_sh;
   float* lse;
@@ -83,12 +84,24 @@ struct FwdArgs {
   CUtensorMap tm_q, tm_k, tm_v;
 };
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t s);
-size_t fwd_varlen_workspace_bytes(int n_seq);
+
+// ---- packed variable-length batches ----
+// Bytes of the sequence table (3 n_seq + 1 int32, 256-aligned) and the kernel that writes it
+// from cu_seqlens (device int32 [n_seq + 1]).
+inline size_t seq_table_bytes(int n_seq) { return align_up((size_t)(3 * n_seq + 1) * sizeof(int32_t), 256); }
+cudaError_t launch_seq_table(const int32_t* cu_seqlens, int n_seq, int total, int32_t* tab, cudaStream_t s);
+// upper bound on the 128-row tiles of a packed batch: sum of ceil(len / 128) <= total / 128 + n_seq
+inline long long packed_tiles_bound(int total, int n_seq) { return (long long)total / 128 + n_seq; }
 
 // ---- backward ----
 struct BwdArgs {
   Pat pat;
   int B, N, Hq, Hkv, d;
+  // packed variable-length batch (varlen != 0, B = 1): the sequences of seq_tab (see
+  // kernel_common.cuh) on a token axis of `total` rows; N is then unused
+  int varlen, n_seq, total;
+  int32_t* seq_tab;
+  int lse_ld;        // row stride of lse: N ([B, Hq, N]) or total (packed: [Hq, total])
   const void* o; int64_t o_sb, o_st, o_sh;
   const void* dO; int64_t do_sb, do_st, do_sh;
   const float* lse;
@@ -97,7 +110,8 @@ struct BwdArgs {
   void* dv; int64_t dv_sb, dv_st, dv_sh;
   float* delta;      // [B, Hq, N_pad] fp32 workspace: rowsum(dO * O), 0 on padded rows
   float* lse2;       // [B, Hq, N_pad] fp32 workspace: lse * log2(e), +inf on padded rows
-  int N_pad;         // N rounded up to a whole number of 128-row tiles
+  int N_pad;         // N rounded up to a whole number of 128-row tiles (packed: 128 x the
+                     // tile bound, each sequence's rows starting at its own tile)
   uint32_t* status;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)

@@ -31,6 +31,22 @@ struct TileCursor {
   }
 };
 
+// Packed variable-length batches.  A sequence table in device memory, written by the
+// seq_table kernel (launch_seq_table) from the caller's cu_seqlens, n = number of sequences:
+//   tab[0 .. n]          tiles of 128 rows before sequence s (tab[n]: all tiles)
+//   tab[n+1 .. 2n]       first row of sequence s on the packed token axis
+//   tab[2n+1 .. 3n]      length of sequence s
+// The offsets are clamped so that the sequences lie in order, disjoint, inside [0, total):
+// start = clamp(cu[s], end of s-1, total), end = clamp(cu[s+1], start, total).
+__device__ __forceinline__ int seq_of_tile(const int32_t* tab, int n, int tg) {
+  int lo = 0, hi = n - 1;  // largest s with tab[s] <= tg (empty sequences share their offset)
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab[mid] <= tg) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }

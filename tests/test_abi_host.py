@@ -270,29 +270,32 @@ def test_fwd_varlen_rejects_bad_arguments_before_launch():
                              n, None) == 1                                                          # no sequences
 
 
-def test_bwd_varlen_rejects_bad_offsets_before_launch():
-    """Host cu_seqlens are checked (start 0, non-decreasing, end = total, lengths <= max_len)
-    before anything is enqueued; the workspace grows with max_len."""
+def test_bwd_varlen_rejects_bad_arguments_before_launch():
+    """The packed backward takes device cu_seqlens like the packed forward: the host checks what
+    it can see (counts, pointers, alignment, workspace size) before anything is enqueued; the
+    workspace holds the sequence table and the statistics of total/128 + n_seq tiles."""
     L = cw.lib()
     p = cw.Pattern(64, 8, 1024, 4).c()
-    n = L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 600, 8, 4, 128)
-    assert n >= L.cowa_bwd_workspace_size(ctypes.byref(p), 1, 600, 8, 4, 128) + 8 * 600 * 4
-    assert L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 1200, 8, 4, 128) > n
-    assert L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 600, 8, 4, 96) == 0
+    n = L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 3, 1000, 8, 4, 128)
+    tiles = 1000 // 128 + 3
+    assert n >= 256 + 4 * (3 * 3 + 1) + 2 * 8 * tiles * 128 * 4
+    assert L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 6, 1000, 8, 4, 128) > n
+    assert L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 3, 1000, 8, 4, 96) == 0
+    assert L.cowa_bwd_varlen_workspace_size(ctypes.byref(p), 0, 1000, 8, 4, 128) == 0
+    args = (ctypes.byref(p), 3, 1000, 8, 4, 128)
 
-    def call(cu, total=1000, max_len=600, lse=0x20000, ws_bytes=n):
-        arr = np.asarray(cu, dtype=np.int32)
-        return L.cowa_bwd_varlen(ctypes.byref(p), len(cu) - 1, arr.ctypes.data_as(ctypes.c_void_p), total, max_len,
-                                 8, 4, 128, _t(), _t(), _t(), _t(), lse, _t(), _t(), _t(), _t(), 0x40000, ws_bytes,
-                                 None)
-    assert call([1, 400, 1000]) == 1                    # does not start at 0
-    assert call([0, 400, 999]) == 1                     # does not end at total
-    assert call([0, 500, 400, 1000]) == 1               # decreasing
-    assert call([0, 700, 1000]) == 4                    # a length above max_len
-    assert call([0, 400, 1000], lse=0x20002) == 3       # misaligned lse
-    assert call([0, 400, 1000], ws_bytes=n - 1) == 4    # small workspace
-    assert L.cowa_bwd_varlen(ctypes.byref(p), 2, None, 1000, 600, 8, 4, 128, _t(), _t(), _t(), _t(), 0x20000,
-                             _t(), _t(), _t(), _t(), 0x40000, n, None) == 1
+    def call(cu=0x30000, lse=0x20000, ws_bytes=n, n_seq=3):
+        return L.cowa_bwd_varlen(ctypes.byref(p), n_seq, 1000, 8, 4, 128, cu, _t(), _t(), _t(), _t(), lse, _t(),
+                                 _t(), _t(), _t(), 0x40000, ws_bytes, None)
+    assert call(cu=None) == 1                 # no cu_seqlens
+    assert call(cu=0x30002) == 3              # misaligned cu_seqlens
+    assert call(lse=None) == 1                # no lse
+    assert call(lse=0x20002) == 3             # misaligned lse
+    assert call(ws_bytes=n - 1) == 4          # small workspace
+    assert call(n_seq=0) == 1                 # no sequences
+    bad = cw.c_tensor(0x10004, 1 << 20, 1024, 128)
+    assert L.cowa_bwd_varlen(*args, 0x30000, _t(), _t(), _t(), _t(), 0x20000, bad, _t(), _t(), _t(), 0x40000, n,
+                             None) == 3       # misaligned dO
 
 
 def test_decode_and_bwd_reject_bad_arguments():

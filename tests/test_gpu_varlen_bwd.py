@@ -1,5 +1,6 @@
-"""GPU parity: the backward of a packed variable-length batch (cowa_bwd_varlen, host cu_seqlens)
-against the fp64 oracle's backward over each sequence alone.
+"""GPU parity: the backward of a packed variable-length batch (cowa_bwd_varlen: device cu_seqlens,
+one launch per backward kernel over all sequences) against the fp64 oracle's backward over each
+sequence alone.
 
 Tolerance: relative Frobenius error <= 1e-2 for dq, dk, dv per sequence, as for cowa_bwd; the
 length-1 sequence has dq = dk = 0 exactly and is judged by its absolute error (gpu_helpers.VANISH).
@@ -20,6 +21,7 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("Hq,Hkv,d,pat,lens", [
     (10, 2, 128, cw.Pattern(32, 200, 1000, 2), [1, 127, 0, 128, 300, 1000]),   # group of 5, an empty sequence
     (8, 4, 128, cw.Pattern(0, 40, 500, 4), [129, 257, 64]),                     # no sink, group of 2
+    (4, 2, 64, cw.Pattern(8, 30, 200, 2), [int(x) for x in np.random.default_rng(3).integers(1, 150, 64)]),  # 64 short
 ])
 def test_bwd_varlen_packed_batch(cuda_device, Hq, Hkv, d, pat, lens):
     total = sum(lens)
@@ -28,8 +30,9 @@ def test_bwd_varlen_packed_batch(cuda_device, Hq, Hkv, d, pat, lens):
     v64, v = host_and_device((1, total, Hkv, d), "v", cuda_device, 37)
     do64, do = host_and_device((1, total, Hq, d), "do", cuda_device, 37)
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    o, lse = cw.cowa_fwd_varlen(q[0], k[0], v[0], torch.tensor(cu, device=cuda_device), pat)
-    dq, dk, dv = cw.cowa_bwd_varlen(q[0], k[0], v[0], o, lse, do[0], cu, pat)
+    cu_d = torch.tensor(cu, device=cuda_device)
+    o, lse = cw.cowa_fwd_varlen(q[0], k[0], v[0], cu_d, pat)
+    dq, dk, dv = cw.cowa_bwd_varlen(q[0], k[0], v[0], o, lse, do[0], cu_d, pat)
     torch.cuda.synchronize()
     op = oracle_pattern(pat)
     report = []
