@@ -37,13 +37,20 @@ constexpr int kDecWarps = 4;                        // compute warps per CTA
 constexpr int kDecThreads = (kDecWarps + 1) * 32;   // + one TMA producer warp
 constexpr int kSubTok = 64;                         // tokens per sub-tile (TMA box rows)
 constexpr int kStages = 3;                          // sub-tile ring depth (bf16 cache)
-constexpr int kMaxStages = 4;                       // ring depth of the E4M3 cache (half-size stages)
+constexpr int kMaxStages = 6;                       // ring depth of the E4M3 cache (half-size stages)
 constexpr int kBoxBytes = kSubTok * 128;            // one [64 rows x 64 bf16] box
 constexpr float kDecRescale = 8.0f;                 // lazy-rescale threshold, log2 units
 
-// KV8: the cache holds E4M3 codes (one byte per element) instead of bf16; each compute warp
-// widens its 16 token rows of a sub-tile to f16 in a scratch tile of its own and runs the same
-// MMAs in f16 (E4M3 values are exact in f16).
+// KV8: the cache holds E4M3 codes (one byte per element) instead of bf16.  Each compute thread
+// loads the code bytes its MMA fragments need straight from the ring into registers and widens
+// them there to f16 (E4M3 values are exact in f16); the MMAs then run in f16.  To make those
+// bytes contiguous, the head dimension is visited in a permuted order (a sum over d, and a
+// relabelling of the output columns, so the result is unchanged):
+//   scores: k-chunk c, in-chunk index kappa of the m16n8k16 operands  <->  d = 32 t + 4 c + j,
+//           t = (kappa mod 8) / 2, j = (kappa mod 2) + 2 [kappa >= 8]  (thread t reads bytes
+//           [32 t, 32 t + 32) of a key row; the query fragments are gathered to match);
+//   P.V:    n-tile jn, column nu  <->  d = 16 nu + jn  (thread g of an MMA group reads bytes
+//           [16 g, 16 g + 16) of each of its 4 value rows), undone when the output is stored.
 template <int D, bool KV8 = false>
 struct DecGeom {
   static_assert(!KV8 || D == 128, "the E4M3 cache needs whole 128-byte rows (d = 128)");
@@ -53,15 +60,8 @@ struct DecGeom {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kStages = KV8 ? kMaxStages : ::cowa::kStages;
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kWarpScratch = KV8 ? 2 * (D / 64) * 16 * 128 : 0;  // f16 K and V, 16 rows
-  static constexpr int kSmemBytes = kRingBytes + kDecWarps * kWarpScratch + 1024;
+  static constexpr int kSmemBytes = kRingBytes + 1024;
 };
-
-// shared address of 16-byte unit u (8 halves: d = 8u..8u+7) of row r of a 16-row f16 tile in the
-// same swizzled form as a TMA tile (128-byte rows, 16-row boxes of 64 halves)
-__device__ __forceinline__ uint32_t unit_addr16(uint32_t tile, int r, int u) {
-  return tile + (u >> 3) * (16 * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-}
 
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   // the low byte becomes the low half
@@ -97,8 +97,10 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
 }
 
 // shared address of 16-byte unit u (d elements 8u..8u+7) of token row r of a swizzled tile
@@ -112,7 +114,7 @@ __device__ __forceinline__ float safe_ex2_diff(float a, float m) {
 }
 
 template <int GRP, int D, bool KV8>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+__device__ __forceinline__ void decode_split_body(const DecodeArgs& a) {
   static_assert(GRP >= 1 && GRP <= 8, "query heads per KV head must fit the MMA's first 8 rows");
   using Geo = DecGeom<D, KV8>;
   constexpr int KS = D / 16;  // k-steps of the score MMA
@@ -227,17 +229,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         reinterpret_cast<const __nv_bfloat16*>(a.q_t) + ((size_t)b * a.Hq + (size_t)g * GRP + imin(gr, GRP - 1)) * D);
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
-      qa[kk][0] = gr < GRP ? qrow[8 * kk + tq] : 0u;
-      qa[kk][1] = gr < GRP ? qrow[8 * kk + 4 + tq] : 0u;
-      if constexpr (KV8) {  // f16 operands (bf16 values of the usual range are exact in f16)
-        qa[kk][0] = bf16x2_to_f16x2(qa[kk][0]);
-        qa[kk][1] = bf16x2_to_f16x2(qa[kk][1]);
+      if constexpr (KV8) {
+        // permuted k order (see DecGeom): chunk kk of thread tq is d = 32 tq + 4 kk .. + 3; f16
+        // operands (bf16 values of the usual range are exact in f16)
+        qa[kk][0] = gr < GRP ? bf16x2_to_f16x2(qrow[16 * tq + 2 * kk]) : 0u;
+        qa[kk][1] = gr < GRP ? bf16x2_to_f16x2(qrow[16 * tq + 2 * kk + 1]) : 0u;
+      } else {
+        qa[kk][0] = gr < GRP ? qrow[8 * kk + tq] : 0u;
+        qa[kk][1] = gr < GRP ? qrow[8 * kk + 4 + tq] : 0u;
       }
     }
   }
-  // this warp's f16 scratch tiles (E4M3 cache only)
-  const uint32_t ksc = ptx::smem_u32(smem) + Geo::kRingBytes + warp * Geo::kWarpScratch;
-  const uint32_t vsc = ksc + Geo::kWarpScratch / 2;
   float acc[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
@@ -251,39 +253,48 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     if (!ptx::mbar_wait_warp(&full_bar[s], (st / kStages) & 1, &abort_flag, a.status)) { ok = false; break; }
     const uint32_t kt = smem_base + s * Geo::kStageBytes;
     const uint32_t vt = kt + Geo::kTileBytes;
-    if constexpr (KV8) {
-      // widen this warp's 16 rows of the E4M3 K and V sub-tiles (128-byte swizzled rows, unit u =
-      // codes of d = 16u..16u+15) to f16 (units 2u, 2u+1 of the scratch row); then the stage is free
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int x = it * 32 + lane;          // 0..255: {K, V} x 16 rows x 8 units
-        const int which = x >> 7, r = (x >> 3) & 15, u = x & 7;
-        const int rr = row0 + r;
-        const uint4 raw = lds128((which ? vt : kt) + rr * 128 + ((u ^ (rr & 7)) << 4));
-        const uint32_t dst = which ? vsc : ksc;
-        sts128(unit_addr16(dst, r, 2 * u), e4m3x2_to_f16x2(raw.x & 0xffffu), e4m3x2_to_f16x2(raw.x >> 16),
-               e4m3x2_to_f16x2(raw.y & 0xffffu), e4m3x2_to_f16x2(raw.y >> 16));
-        sts128(unit_addr16(dst, r, 2 * u + 1), e4m3x2_to_f16x2(raw.z & 0xffffu), e4m3x2_to_f16x2(raw.z >> 16),
-               e4m3x2_to_f16x2(raw.w & 0xffffu), e4m3x2_to_f16x2(raw.w >> 16));
-      }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
-    }
     // ---- scores S[head][token] for two 8-token n-tiles
     float sc[2][4];
+    uint4 vr[4];  // E4M3 only: bytes [16 gr, 16 gr + 16) of value rows 2tq, 2tq+1, 2tq+8, 2tq+9
+    if constexpr (KV8) {
+      // key codes straight into registers: thread tq takes bytes [32 tq, 32 tq + 32) of key row
+      // 8 nt + gr (two 16-byte units of the swizzled row), which are its B fragments of all 8
+      // k-chunks in the permuted order; value codes likewise (see DecGeom)
+      uint32_t kw[2][8];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      for (int nt = 0; nt < 2; ++nt) {
+        const int r = row0 + 8 * nt + gr;
+        const uint32_t rb = kt + r * 128;
+        const uint4 x0 = lds128(rb + (((2 * tq) ^ (r & 7)) << 4));
+        const uint4 x1 = lds128(rb + (((2 * tq + 1) ^ (r & 7)) << 4));
+        kw[nt][0] = x0.x; kw[nt][1] = x0.y; kw[nt][2] = x0.z; kw[nt][3] = x0.w;
+        kw[nt][4] = x1.x; kw[nt][5] = x1.y; kw[nt][6] = x1.z; kw[nt][7] = x1.w;
+      }
 #pragma unroll
-      for (int k2 = 0; k2 < KS / 2; ++k2) {
-        uint32_t bb[4];
-        const uint32_t a0[4] = {qa[2 * k2][0], 0u, qa[2 * k2][1], 0u};
-        const uint32_t a1[4] = {qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u};
-        if constexpr (KV8) {
-          ptx::ldsm_x4(unit_addr16(ksc, 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
-          mma_16816_f16(sc[nt], a0, bb[0], bb[1]);
-          mma_16816_f16(sc[nt], a1, bb[2], bb[3]);
-        } else {
+      for (int i = 0; i < 4; ++i) {
+        const int r = row0 + 2 * tq + (i & 1) + 8 * (i >> 1);
+        vr[i] = lds128(vt + r * 128 + ((gr ^ (r & 7)) << 4));
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);  // the stage's bytes are in registers
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const uint32_t aa[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+          mma_16816_f16(sc[nt], aa, e4m3x2_to_f16x2(kw[nt][kk] & 0xffffu), e4m3x2_to_f16x2(kw[nt][kk] >> 16));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int k2 = 0; k2 < KS / 2; ++k2) {
+          uint32_t bb[4];
+          const uint32_t a0[4] = {qa[2 * k2][0], 0u, qa[2 * k2][1], 0u};
+          const uint32_t a1[4] = {qa[2 * k2 + 1][0], 0u, qa[2 * k2 + 1][1], 0u};
           ptx::ldsm_x4(unit_addr(kt, row0 + 8 * nt + (lane & 7), 4 * k2 + (lane >> 3)), bb);
           ptx::mma_16816(sc[nt], a0, bb[0], bb[1]);
           ptx::mma_16816(sc[nt], a1, bb[2], bb[3]);
@@ -325,21 +336,33 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     }
     pa[1] = pa[3] = 0u;
     // ---- O[head][d] += P[head][token] V[token][d]
+    if constexpr (KV8) {
+      // n-tile jn, column gr is d = 16 gr + jn: byte jn of this thread's value bytes.  Bytes of
+      // rows (2tq, 2tq+1) and (2tq+8, 2tq+9) are interleaved into E4M3 pairs, then widened.
+      const uint32_t A[4] = {vr[0].x, vr[0].y, vr[0].z, vr[0].w}, B[4] = {vr[1].x, vr[1].y, vr[1].z, vr[1].w};
+      const uint32_t C[4] = {vr[2].x, vr[2].y, vr[2].z, vr[2].w}, E[4] = {vr[3].x, vr[3].y, vr[3].z, vr[3].w};
 #pragma unroll
-    for (int np = 0; np < NT / 2; ++np) {
-      uint32_t bb[4];
-      if constexpr (KV8) {
-        ptx::ldsm_x4_trans(unit_addr16(vsc, (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
-        mma_16816_f16(acc[2 * np], pa, bb[0], bb[1]);
-        mma_16816_f16(acc[2 * np + 1], pa, bb[2], bb[3]);
-      } else {
+      for (int jw = 0; jw < 4; ++jw) {
+        const uint32_t ab[2] = {prmt(A[jw], B[jw], 0x5140u), prmt(A[jw], B[jw], 0x7362u)};
+        const uint32_t ce[2] = {prmt(C[jw], E[jw], 0x5140u), prmt(C[jw], E[jw], 0x7362u)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int sh = (e & 1) * 16;
+          mma_16816_f16(acc[4 * jw + e], pa, e4m3x2_to_f16x2((ab[e >> 1] >> sh) & 0xffffu),
+                        e4m3x2_to_f16x2((ce[e >> 1] >> sh) & 0xffffu));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        uint32_t bb[4];
         ptx::ldsm_x4_trans(unit_addr(vt, row0 + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * np + (lane >> 4)), bb);
         ptx::mma_16816(acc[2 * np], pa, bb[0], bb[1]);
         ptx::mma_16816(acc[2 * np + 1], pa, bb[2], bb[3]);
       }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty_bar[s]);
     }
-    __syncwarp();  // (KV8: the scratch is rewritten by the next sub-tile's widening)
-    if (!KV8 && lane == 0) ptx::mbar_arrive(&empty_bar[s]);
   }
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
   lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
@@ -353,8 +376,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     if (tq == 0) { rw[0] = m_used; rw[1] = lsum; }
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      rw[2 + 8 * n + 2 * tq] = acc[n][0];
-      rw[2 + 8 * n + 2 * tq + 1] = acc[n][1];
+      if constexpr (KV8) {  // columns 2tq, 2tq+1 of n-tile n are d = 32 tq + n and 32 tq + 16 + n
+        rw[2 + 32 * tq + n] = acc[n][0];
+        rw[2 + 32 * tq + 16 + n] = acc[n][1];
+      } else {
+        rw[2 + 8 * n + 2 * tq] = acc[n][0];
+        rw[2 + 8 * n + 2 * tq + 1] = acc[n][1];
+      }
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kDecWarps * 32) : "memory");
@@ -376,6 +404,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     out[2 + dc] = KV8 ? o * a.v_scale : o;
     if (dc == 0) { out[0] = mxw; out[1] = ll; }
   }
+}
+
+// bf16 cache
+template <int GRP, int D>
+__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeArgs a) {
+  decode_split_body<GRP, D, false>(a);
+}
+// E4M3 cache: two CTAs per SM (6-stage ring, no register spills)
+template <int GRP>
+__global__ void __launch_bounds__(kDecThreads, 2) decode_split_e4m3_kernel(const __grid_constant__ DecodeArgs a) {
+  decode_split_body<GRP, 128, true>(a);
 }
 
 // One warp per (b, h): merge the n_split partial states, write bf16 o and fp32 lse.
@@ -465,7 +504,9 @@ __global__ void __launch_bounds__(128) compact_build_kernel(Pat pat, CompactGeom
 template <int GRP, int D, bool KV8>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
   using Geo = DecGeom<D, KV8>;
-  auto kern = decode_split_kernel<GRP, D, KV8>;
+  void (*kern)(const DecodeArgs);
+  if constexpr (KV8) kern = decode_split_e4m3_kernel<GRP>;
+  else kern = decode_split_kernel<GRP, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_split, a.Hkv, a.B);

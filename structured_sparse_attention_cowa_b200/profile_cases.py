@@ -1,12 +1,14 @@
 """Small, fixed invocations of each hot kernel for profiling with ncu.
 
-    python -m structured_sparse_attention_cowa_b200.profile_cases {fwd32k,bwd32k,decode128k_b4,all} [--reps R]
+    python -m structured_sparse_attention_cowa_b200.profile_cases {fwd32k,bwd32k,decode128k_b4,decode128k_e4m3_b4,all}
+        [--reps R]
 
 Each case allocates its seeded inputs on cuda:0 (a few GB at most), calls the C ABI
 `reps` times (the first launch warms up; profile with `-s 1 -c 1` on the kernel name) and
 checks the device status word.  Shapes follow the 32K training layer (B=1, N=32768,
 H_q=40, H_kv=8, d=128, S=128, L=2048, D=8) and the 128K decode cache at 4 sequences
-(H_q=40, H_kv=8, d=128, T_cap=131072, pos=131071, S=128, L=4096, D=8).
+(H_q=40, H_kv=8, d=128, T_cap=131072, pos=131071, S=128, L=4096, D=8), in bf16 or quantised to
+E4M3 (scale 1/64).
 """
 
 from __future__ import annotations
@@ -71,7 +73,25 @@ def case_decode128k_b4(dev, reps):
     return [ws]
 
 
-CASES = {"fwd32k": case_fwd32k, "bwd32k": case_bwd32k, "decode128k_b4": case_decode128k_b4}
+def case_decode128k_e4m3_b4(dev, reps):
+    B, Hq, Hkv, d, Tc = 4, 40, 8, 128, 131072
+    pat = cw.Pattern(128, 4096, 131072, 8)
+    scale = 1.0 / 64
+    kc = cw.quantize_e4m3(synth.cuda_normal_bf16((B, Hkv, Tc, d), synth.seed_of("k_cache"), dev), scale)
+    vc = cw.quantize_e4m3(synth.cuda_normal_bf16((B, Hkv, Tc, d), synth.seed_of("v_cache"), dev), scale)
+    qt = synth.cuda_normal_bf16((B, Hq, d), synth.seed_of("q_t"), dev)
+    pos = torch.full((B,), Tc - 1, dtype=torch.int32, device=dev)
+    import ctypes
+
+    n = cw.lib().cowa_decode_fp8_workspace_size(ctypes.byref(pat.c()), B, Hq, Hkv, d, Tc)
+    ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    for _ in range(reps):
+        cw.cowa_decode_fp8(qt, kc, vc, pos, pat, scale, scale, workspace=ws)
+    return [ws]
+
+
+CASES = {"fwd32k": case_fwd32k, "bwd32k": case_bwd32k, "decode128k_b4": case_decode128k_b4,
+         "decode128k_e4m3_b4": case_decode128k_e4m3_b4}
 
 
 def main(argv=None):
