@@ -52,24 +52,35 @@ COWA_HD bool visible(const Pat& p, Range iv, int t, int s) {
 }
 
 // Sort up to three ranges by lo, drop empty ones and merge overlapping or
-// touching ones.  Returns the number of disjoint ranges written to r[0..n).
+// touching ones.  Returns the number n of disjoint ranges written to r[0..n);
+// r[n..3) are set to the empty sentinel [INT_MAX, INT_MAX).  Written with fixed
+// indices only, so that a kernel keeps everything in registers.
 COWA_HD int merge3(Range a, Range b, Range c, Range* r) {
-  Range v[3] = {a, b, c};
+  constexpr int kNone = 0x7fffffff;
+  Range v0 = a, v1 = b, v2 = c;
   // 3-element sorting network on lo (empty ranges pushed last by lo = INT_MAX)
-  for (int i = 0; i < 3; ++i)
-    if (v[i].lo >= v[i].hi) { v[i].lo = 0x7fffffff; v[i].hi = 0x7fffffff; }
-  if (v[1].lo < v[0].lo) { Range x = v[0]; v[0] = v[1]; v[1] = x; }
-  if (v[2].lo < v[1].lo) { Range x = v[1]; v[1] = v[2]; v[2] = x; }
-  if (v[1].lo < v[0].lo) { Range x = v[0]; v[0] = v[1]; v[1] = x; }
-  int n = 0;
-  for (int i = 0; i < 3; ++i) {
-    if (v[i].lo == 0x7fffffff) break;
-    if (n > 0 && v[i].lo <= r[n - 1].hi) {
-      r[n - 1].hi = imax(r[n - 1].hi, v[i].hi);
+  if (v0.lo >= v0.hi) { v0.lo = kNone; v0.hi = kNone; }
+  if (v1.lo >= v1.hi) { v1.lo = kNone; v1.hi = kNone; }
+  if (v2.lo >= v2.hi) { v2.lo = kNone; v2.hi = kNone; }
+  if (v1.lo < v0.lo) { Range x = v0; v0 = v1; v1 = x; }
+  if (v2.lo < v1.lo) { Range x = v1; v1 = v2; v2 = x; }
+  if (v1.lo < v0.lo) { Range x = v0; v0 = v1; v1 = x; }
+  Range o0 = v0, o1{kNone, kNone}, o2{kNone, kNone};
+  int n = v0.lo != kNone ? 1 : 0;
+  if (v1.lo != kNone) {
+    if (v1.lo <= o0.hi) o0.hi = imax(o0.hi, v1.hi);
+    else { o1 = v1; n = 2; }
+  }
+  if (v2.lo != kNone) {
+    if (n == 1) {
+      if (v2.lo <= o0.hi) o0.hi = imax(o0.hi, v2.hi);
+      else { o1 = v2; n = 2; }
     } else {
-      r[n++] = v[i];
+      if (v2.lo <= o1.hi) o1.hi = imax(o1.hi, v2.hi);
+      else { o2 = v2; n = 3; }
     }
   }
+  r[0] = o0; r[1] = o1; r[2] = o2;
   return n;
 }
 

@@ -9,25 +9,35 @@ namespace cowa {
 constexpr int kTile = 128;  // query and key tile edge (BM = BN = 128)
 
 struct Tiles {
-  Range r[3];
-  int n;      // number of disjoint tile-index ranges
-  int count;  // number of tiles
+  Range r[3];  // disjoint tile-index ranges r[0..n); the rest are empty sentinels
+  int n;       // number of ranges
+  int count;   // number of tiles
 };
 
 __device__ __forceinline__ Tiles plan_tiles(const Pat& p, Range iv, int t0, int t1) {
   Tiles T;
   T.n = fwd_tile_ranges(p, iv, t0, t1, kTile, T.r);
-  T.count = 0;
-  for (int x = 0; x < T.n; ++x) T.count += T.r[x].hi - T.r[x].lo;
+  // fixed indices only (the sentinels [INT_MAX, INT_MAX) count 0), so T stays in registers
+  T.count = (T.r[0].hi - T.r[0].lo) + (T.r[1].hi - T.r[1].lo) + (T.r[2].hi - T.r[2].lo);
   return T;
 }
 
-// Walks the tile list in order.
+// Walks the tile list in order, in registers: the current tile, the end of its range and the
+// ranges still to come (no array indexed at run time, which would live in local memory).
 struct TileCursor {
-  int x, j;
-  __device__ __forceinline__ void init(const Tiles& T) { x = 0; j = T.n > 0 ? T.r[0].lo : 0; }
-  __device__ __forceinline__ void next(const Tiles& T) {
-    if (++j >= T.r[x].hi && x + 1 < T.n) { ++x; j = T.r[x].lo; }
+  int j, hi, lo1, hi1, lo2, hi2;
+  __device__ __forceinline__ void init(const Tiles& T) {
+    j = T.n > 0 ? T.r[0].lo : 0;
+    hi = T.n > 0 ? T.r[0].hi : 0;
+    lo1 = T.r[1].lo; hi1 = T.r[1].hi;
+    lo2 = T.r[2].lo; hi2 = T.r[2].hi;
+  }
+  __device__ __forceinline__ void next(const Tiles&) {
+    if (++j >= hi && lo1 != 0x7fffffff) {
+      j = lo1; hi = hi1;
+      lo1 = lo2; hi1 = hi2;
+      lo2 = 0x7fffffff; hi2 = 0x7fffffff;
+    }
   }
 };
 
