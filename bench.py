@@ -308,7 +308,8 @@ def config_parts(dev, kc, vc, peak_tf, hbm_gbs, sweep=False, reps=2):
     layer itself, its dense-causal mode (L >= T, the FullAttn comparison) and SWA + sinks
     (T = S), the 128K layer and its dense-causal mode, and the 128K decode over the full
     cache, in the dense-causal mode, over the compacted cache and over E4M3 caches; `sweep`
-    adds the 8K prefill D sweep.  Returns {key: row}."""
+    adds the 8K prefill D sweep.  The decodes run first (before the long training kernels warm the
+    GPU into its power-capped state).  Returns {key: row}."""
     import ctypes
 
     import torch
@@ -333,48 +334,6 @@ def config_parts(dev, kc, vc, peak_tf, hbm_gbs, sweep=False, reps=2):
             b.record(); torch.cuda.synchronize()
             ts.append(a.elapsed_time(b) / inner)
         return statistics.median(ts)
-
-    for key, B, N, Hq, Hkv, d, S, L, T, D, do_bwd, default in CONFIGS:
-        if not (default or sweep):
-            continue
-        pat = cw.Pattern(S, L, T, D)
-        q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), dev)
-        k = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("k"), dev)
-        v = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("v"), dev)
-        o = torch.empty_like(q)
-        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
-        n_ws = cw.lib().cowa_fwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
-        ws_f = torch.zeros(max(256, n_ws), dtype=torch.uint8, device=dev)
-        pairs = visible_pairs(N, S, L, T, D, Hkv, Hq, B)
-        f_ms = timed(lambda: cw.cowa_fwd(q, k, v, pat, out=o, lse=lse, workspace=ws_f))
-        row = {"B": B, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "S": S, "L": L, "T": T, "D": D,
-               "visible_pairs": pairs, "fwd_ms": f_ms, "fwd_tflops": 4.0 * d * pairs / (f_ms * 1e-3) / 1e12}
-        row["fwd_frac_burst"] = row["fwd_tflops"] / peak_tf
-        if do_bwd:
-            do = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("do"), dev)
-            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-            n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
-            ws = torch.zeros(n, dtype=torch.uint8, device=dev)
-            stage = lambda st: cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws, stages=st)
-            st_ms = {nm: timed(lambda st=st: stage(st)) for nm, st in
-                     (("preprocess", cw.BWD_PREPROCESS), ("dkdv", cw.BWD_DKDV), ("dq", cw.BWD_DQ))}
-            b_ms = sum(st_ms.values())
-            row.update({"bwd_ms": b_ms, "bwd_stages_ms": st_ms, "bwd_tflops": 10.0 * d * pairs / (b_ms * 1e-3) / 1e12})
-            row["bwd_frac_burst"] = row["bwd_tflops"] / peak_tf
-            if cw.workspace_status(ws) != 0:
-                raise RuntimeError(f"device status set in configuration {key}")
-            del do, dq, dk, dv, ws
-        if cw.workspace_status(ws_f) != 0:
-            raise RuntimeError(f"device status set in configuration {key}")
-        out[key] = row
-        del q, k, v, o, lse, ws_f
-        torch.cuda.empty_cache()
-    for key in ("train_32k_dense_causal", "long_128k_dense_causal"):
-        base = key.replace("_dense_causal", "")
-        if key in out and base in out:  # CoWA against the dense-causal mode of the same kernels
-            out[key]["cowa_fwd_speedup"] = out[key]["fwd_ms"] / out[base]["fwd_ms"]
-            if "bwd_ms" in out[key] and "bwd_ms" in out[base]:
-                out[key]["cowa_bwd_speedup"] = out[key]["bwd_ms"] / out[base]["bwd_ms"]
 
     # decode at 128K (B = 16, pos = 131071): the CoWA pattern over the full cache, the
     # dense-causal mode (every cached token up to pos visible), the CoWA pattern over the
@@ -437,6 +396,49 @@ def config_parts(dev, kc, vc, peak_tf, hbm_gbs, sweep=False, reps=2):
         if cw.workspace_status(w) != 0:
             raise RuntimeError("device status set in the decode configurations")
     torch.cuda.empty_cache()
+
+    for key, B, N, Hq, Hkv, d, S, L, T, D, do_bwd, default in CONFIGS:
+        if not (default or sweep):
+            continue
+        pat = cw.Pattern(S, L, T, D)
+        q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), dev)
+        k = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("k"), dev)
+        v = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("v"), dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        n_ws = cw.lib().cowa_fwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+        ws_f = torch.zeros(max(256, n_ws), dtype=torch.uint8, device=dev)
+        pairs = visible_pairs(N, S, L, T, D, Hkv, Hq, B)
+        f_ms = timed(lambda: cw.cowa_fwd(q, k, v, pat, out=o, lse=lse, workspace=ws_f))
+        row = {"B": B, "N": N, "Hq": Hq, "Hkv": Hkv, "d": d, "S": S, "L": L, "T": T, "D": D,
+               "visible_pairs": pairs, "fwd_ms": f_ms, "fwd_tflops": 4.0 * d * pairs / (f_ms * 1e-3) / 1e12}
+        row["fwd_frac_burst"] = row["fwd_tflops"] / peak_tf
+        if do_bwd:
+            do = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("do"), dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+            ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+            stage = lambda st: cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv, workspace=ws, stages=st)
+            st_ms = {nm: timed(lambda st=st: stage(st)) for nm, st in
+                     (("preprocess", cw.BWD_PREPROCESS), ("dkdv", cw.BWD_DKDV), ("dq", cw.BWD_DQ))}
+            b_ms = sum(st_ms.values())
+            row.update({"bwd_ms": b_ms, "bwd_stages_ms": st_ms, "bwd_tflops": 10.0 * d * pairs / (b_ms * 1e-3) / 1e12})
+            row["bwd_frac_burst"] = row["bwd_tflops"] / peak_tf
+            if cw.workspace_status(ws) != 0:
+                raise RuntimeError(f"device status set in configuration {key}")
+            del do, dq, dk, dv, ws
+        if cw.workspace_status(ws_f) != 0:
+            raise RuntimeError(f"device status set in configuration {key}")
+        out[key] = row
+        del q, k, v, o, lse, ws_f
+        torch.cuda.empty_cache()
+    for key in ("train_32k_dense_causal", "long_128k_dense_causal"):
+        base = key.replace("_dense_causal", "")
+        if key in out and base in out:  # CoWA against the dense-causal mode of the same kernels
+            out[key]["cowa_fwd_speedup"] = out[key]["fwd_ms"] / out[base]["fwd_ms"]
+            if "bwd_ms" in out[key] and "bwd_ms" in out[base]:
+                out[key]["cowa_bwd_speedup"] = out[key]["bwd_ms"] / out[base]["bwd_ms"]
+
     return out
 
 
