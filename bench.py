@@ -917,10 +917,37 @@ def run_cowa(args, world, rank, local):
                     if cw.workspace_status(st_[n]) != 0:
                         raise RuntimeError("device status set during the end-to-end steps")
             e_ms = maxr(a.elapsed_time(b)) / KE
+
+            # The same host<->device copies with no kernels between them (copy-in and copy-out on
+            # their own streams, as in the steps above): the PCIe ceiling of this e2e number.
+            def copy_step(i):
+                st = sets[i % 2]
+                with torch.cuda.stream(s_in):
+                    for n in names_in:
+                        st[n].copy_(h_in[n], non_blocking=True)
+                    st["pos"].copy_(h_pos, non_blocking=True)
+                with torch.cuda.stream(s_out):
+                    for n in names_out:
+                        h_out[n].copy_(st[n], non_blocking=True)
+
+            copy_step(0); torch.cuda.synchronize()
+            barrier()
+            a.record(main_s)
+            for st_ in (s_in, s_out):
+                st_.wait_stream(main_s)
+            for i in range(KE):
+                copy_step(i)
+            for st_ in (s_in, s_out):
+                main_s.wait_stream(st_)
+            b.record(main_s); torch.cuda.synchronize()
+            barrier()
+            c_ms = maxr(a.elapsed_time(b)) / KE
             res = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
                    "pipelined": "copy-in / compute / copy-out streams, two device buffer sets",
-                   "outputs_read": list(names_out)}
+                   "outputs_read": list(names_out),
+                   "copy_only_ms_per_step": c_ms, "frac_of_copy_bound": c_ms / e_ms,
+                   "copy_gbs": {"h2d": h2d / c_ms / 1e6, "d2h": d2h / c_ms / 1e6}}
             del sets
             return res
 
@@ -928,7 +955,8 @@ def run_cowa(args, world, rank, local):
         if args.e2e_outputs == "all":
             r = run_e2e(False)
             e2e["results_only"] = {k_: r[k_] for k_ in ("value", "ms_per_step", "h2d_bytes_per_step",
-                                                         "d2h_bytes_per_step", "outputs_read")}
+                                                         "d2h_bytes_per_step", "outputs_read",
+                                                         "copy_only_ms_per_step", "frac_of_copy_bound")}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
