@@ -942,11 +942,15 @@ def run_cowa(args, world, rank, local):
             b.record(main_s); torch.cuda.synchronize()
             barrier()
             c_ms = maxr(a.elapsed_time(b)) / KE
+            # the results that came back to the host equal the device-timed path's, bit for bit
+            # (same inputs, deterministic kernels)
+            match = all(torch.equal(h_out[n].to(dev), dev_out[n]) for n in names_out)
             res = {"value": aggregate_tflops(world, fwd_flop + bwd_flop, e_ms), "unit": "TFLOP/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": KE,
                    "pipelined": "copy-in / compute / copy-out streams, two device buffer sets",
                    "outputs_read": list(names_out),
                    "copy_only_ms_per_step": c_ms, "frac_of_copy_bound": c_ms / e_ms,
+                   "outputs_match_device_path": match,
                    "copy_gbs": {"h2d": h2d / c_ms / 1e6, "d2h": d2h / c_ms / 1e6}}
             del sets
             return res
@@ -956,7 +960,8 @@ def run_cowa(args, world, rank, local):
             r = run_e2e(False)
             e2e["results_only"] = {k_: r[k_] for k_ in ("value", "ms_per_step", "h2d_bytes_per_step",
                                                          "d2h_bytes_per_step", "outputs_read",
-                                                         "copy_only_ms_per_step", "frac_of_copy_bound")}
+                                                         "copy_only_ms_per_step", "frac_of_copy_bound",
+                                                         "outputs_match_device_path")}
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
