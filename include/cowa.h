@@ -57,7 +57,8 @@ typedef enum {
   COWA_OK = 0,
   COWA_ERR_INVALID_ARG = 1, /* bad shape, pattern or null pointer */
   COWA_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128}, or more than 8 query heads per KV
-                               head (H_q / H_kv > 8); the E4M3-cache calls need d = 128 */
+                               head (H_q / H_kv > 8); the E4M3-cache calls need d = 128; a
+                               compacted cache whose rows per head would exceed INT_MAX */
   COWA_ERR_ALIGNMENT = 3,   /* pointer or stride not 16-byte aligned */
   COWA_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
   COWA_ERR_CUDA = 5,        /* CUDA runtime/driver error at launch */
@@ -203,7 +204,8 @@ cowa_status cowa_decode(const cowa_pattern* pat, int B, int H_q, int H_kv, int d
  * At 128K (S=128, L=4096, T=131072, 8 KV heads) that is 20,736 rows per head instead of 131,072.
  * The ring holds the last R positions, so positions must be appended in order (build from a
  * prefill, then one append per decoded token).  The caller owns both arrays. */
-/* Rows per (b, KV head) of the compacted cache; 0 for an invalid pattern. */
+/* Rows per (b, KV head) of the compacted cache; 0 for an invalid pattern or one whose compacted
+ * layout would need more than INT_MAX rows (a band L near INT_MAX: use the full cache). */
 int cowa_compact_rows(const cowa_pattern* pat, int H_kv);
 /* Fills the compacted cache from the keys and values of positions 0..N-1 (k, v as in cowa_fwd:
  * [B, N, H_kv, d] with any cowa_tensor strides).  Rows no position maps to are left untouched. */

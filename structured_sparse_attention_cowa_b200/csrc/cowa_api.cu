@@ -176,6 +176,7 @@ cowa_status cowa_compact_build(const cowa_pattern* pat, int B, int N, int Hkv, i
                                void* k_compact, void* v_compact, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, N, Hkv, Hkv, d));
   COWA_TRY(check_tensor(k));
   COWA_TRY(check_tensor(v));
@@ -192,6 +193,7 @@ cowa_status cowa_compact_append(const cowa_pattern* pat, int B, int Hkv, int d, 
                                 const int32_t* pos, void* k_compact, void* v_compact, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, 1, Hkv, Hkv, d));
   if (!k_new || !v_new || !pos || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_compact) || !aligned16(v_compact))
@@ -215,6 +217,7 @@ cowa_status cowa_decode_compact(const cowa_pattern* pat, int B, int Hq, int Hkv,
                                 float* lse_or_null, void* ws, size_t ws_bytes, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, 1, Hq, Hkv, d));
   if (!q_t || !pos || !o || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
   if (!aligned16(q_t) || !aligned16(o) || !aligned16(k_compact) || !aligned16(v_compact) ||
@@ -327,6 +330,7 @@ cowa_status cowa_compact_build_fp8(const cowa_pattern* pat, int B, int N, int Hk
                                    cowa_tensor v, void* k_compact, void* v_compact, void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, N, Hkv, Hkv, d));
   if (d != 128) return COWA_ERR_UNSUPPORTED;
   COWA_TRY(check_tensor8(k));
@@ -345,6 +349,7 @@ cowa_status cowa_compact_append_fp8(const cowa_pattern* pat, int B, int Hkv, int
                                     void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, 1, Hkv, Hkv, d));
   if (d != 128) return COWA_ERR_UNSUPPORTED;
   if (!k_new || !v_new || !pos || !k_compact || !v_compact) return COWA_ERR_INVALID_ARG;
@@ -366,6 +371,7 @@ cowa_status cowa_decode_fp8_compact(const cowa_pattern* pat, int B, int Hq, int 
                                     void* stream) {
   Pat p;
   COWA_TRY(check_pattern(pat, Hkv, &p));
+  if (compact_geom(p).rows <= 0) return COWA_ERR_UNSUPPORTED;  // layout larger than an int row count
   COWA_TRY(check_heads(B, 1, Hq, Hkv, d));
   if (d != 128) return COWA_ERR_UNSUPPORTED;
   if (!q_t || !pos || !o || !k_compact || !v_compact || !(k_scale > 0.f) || !(v_scale > 0.f) ||

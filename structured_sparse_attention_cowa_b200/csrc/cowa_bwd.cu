@@ -262,7 +262,8 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
     const int s = s0 + r;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const bool special = s < a.pat.S || (s >= iv.lo && s < iv.hi);
-    const int t_hi = special ? N : imin(N, s + a.pat.L);  // rows [s, t_hi) see key s
+    // rows [s, t_hi) see key s (min(N, s + L), without overflow for a window up to INT_MAX)
+    const int t_hi = special ? N : (a.pat.L >= N - s ? N : s + a.pat.L);
     const float sl2 = a.scale_log2;
     bool ok = true;
     // query tile of the current step and its two sub-steps' mask flags, advanced incrementally

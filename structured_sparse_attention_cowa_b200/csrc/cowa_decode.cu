@@ -554,18 +554,25 @@ int decode_num_splits(const Pat& p, int T_cap, int chunk, bool compact) {
   return (int)(n < 1 ? 1 : n);
 }
 
+// Sizes in 64-bit; a layout whose rows would not fit an int (a band of ~2^31 positions) is
+// reported as rows = 0, which the entry points reject.
 CompactGeom compact_geom(const Pat& p) {
-  CompactGeom c;
-  c.S64 = (p.S + kSubTok - 1) / kSubTok * kSubTok;
-  c.R = (p.L + kSubTok - 1) / kSubTok * kSubTok + kSubTok;
-  c.IB = c.S64 + c.R;
-  int w = 0;
+  CompactGeom c{};
+  const int64_t t = kSubTok;
+  const int64_t s64 = ((int64_t)p.S + t - 1) / t * t;
+  const int64_t r = ((int64_t)p.L + t - 1) / t * t + t;
+  int64_t w = 0;
   for (int slot = 0; slot < p.H; slot += p.H / p.D) {  // the distinct interval slots
     const int lo = bound(p, slot), hi = bound(p, slot + 1);
-    if (hi > lo) w = imax(w, hi - (lo & ~(kSubTok - 1)));
+    if (hi > lo) w = w > (int64_t)hi - (lo & ~(kSubTok - 1)) ? w : (int64_t)hi - (lo & ~(kSubTok - 1));
   }
-  c.W = (w + kSubTok - 1) / kSubTok * kSubTok;
-  c.rows = c.IB + c.W;
+  w = (w + t - 1) / t * t;
+  if (s64 + r + w > 0x7fffffffLL) return c;
+  c.S64 = (int)s64;
+  c.R = (int)r;
+  c.IB = (int)(s64 + r);
+  c.W = (int)w;
+  c.rows = (int)(s64 + r + w);
   return c;
 }
 

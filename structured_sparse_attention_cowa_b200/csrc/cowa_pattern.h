@@ -138,7 +138,8 @@ COWA_HD bool tile_full(const Pat& p, Range iv, int t0, int t1, int s0, int s1) {
 COWA_HD Range bwd_row_range(const Pat& p, Range iv, int s0, int s1, int N) {
   // smallest key of the tile that is in the sink or the interval
   bool special = (s0 < p.S) || (iv.lo < iv.hi && iv.lo < s1 && iv.hi > s0);
-  int end = special ? N : imin(N, s1 - 1 + p.L);
+  // band-only: rows up to s1 - 1 + L, written so that a window of up to INT_MAX cannot overflow
+  int end = special ? N : (p.L >= N - s1 + 1 ? N : s1 - 1 + p.L);
   return Range{s0, imax(s0, end)};
 }
 

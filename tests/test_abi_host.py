@@ -38,6 +38,7 @@ def _oracle_pattern(p: cw.Pattern):
 PLAN_CASES = [
     # N, Hkv, BM, BN, pattern
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 4)),       # tiny config
+    (700, 2, 128, 128, cw.Pattern(16, 2**31 - 1, 700, 2)),   # window of INT_MAX (dense causal): no overflow
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 2)),       # duplicated D=2
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 1)),       # duplicated D=1
     (1000, 4, 128, 128, cw.Pattern(64, 128, 1000, 4)),       # ragged tail
@@ -248,6 +249,12 @@ def test_compact_entry_points_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(20, 100, 2000, 2).c()
     assert L.cowa_compact_rows(None, 2) == 0
+    # a band of ~2^31 positions has no compacted layout that an int row count can address
+    wide = cw.Pattern(20, 2**31 - 1, 2000, 2).c()
+    assert L.cowa_compact_rows(ctypes.byref(wide), 2) == 0
+    assert L.cowa_compact_build(ctypes.byref(wide), 2, 100, 2, 128, _t(), _t(), 0x30000, 0x40000, None) == 2
+    assert L.cowa_compact_append(ctypes.byref(wide), 2, 2, 128, 0x10000, 0x20000, 0x50000, 0x30000, 0x40000,
+                                 None) == 2
     assert L.cowa_compact_append(ctypes.byref(p), 2, 2, 128, 0x10000, 0x20000, None, 0x30000, 0x40000, None) == 1
     assert L.cowa_compact_append(ctypes.byref(p), 2, 2, 96, 0x10000, 0x20000, 0x50000, 0x30000, 0x40000, None) == 2
     assert L.cowa_compact_build(ctypes.byref(p), 2, 100, 2, 128, _t(), _t(), 0x30008, 0x40000, None) == 3

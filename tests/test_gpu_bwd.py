@@ -44,6 +44,28 @@ def _check_full(B, N, Hq, Hkv, d, pat, device, extra=0):
     assert max(errs) <= GRAD_RTOL, errs
 
 
+def test_window_of_int_max_equals_dense_causal(cuda_device):
+    """A band of L = INT_MAX (a caller's "no window limit") is the dense-causal mode: forward and
+    backward give the same bits as L = N, and the gradients match the oracle.  The band ends
+    s + L of the backward's row ranges must not overflow (they did before saturating)."""
+    B, N, Hq, Hkv, d = 1, 700, 4, 2, 128
+    host, dev = _inputs(B, N, Hq, Hkv, d, cuda_device, extra=11)
+    wide, dense = cw.Pattern(16, 2**31 - 1, N, 2), cw.Pattern(16, N, N, 2)
+    q, k, v, do = dev
+    o1, l1 = cw.cowa_fwd(q, k, v, wide)
+    o2, l2 = cw.cowa_fwd(q, k, v, dense)
+    g1 = cw.cowa_bwd(q, k, v, o1, l1, do, wide)
+    g2 = cw.cowa_bwd(q, k, v, o2, l2, do, dense)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    op = oracle_pattern(wide)
+    want = orc.attention_bwd(*host, op)
+    errs = grad_errors(tuple(to64(x) for x in g1), want, grad_bounds(*host, op.sm_scale(d)))
+    assert max(errs) <= GRAD_RTOL, errs
+
+
 @pytest.mark.parametrize("D", [4, 2, 1])
 def test_bwd_tiny_config(cuda_device, D):
     """B=1, N=T=1024, H_q=8, H_kv=4, d=64, S=64, L=128; D=4 and the duplicated D=2, 1."""
