@@ -40,7 +40,7 @@ cowa_status check_pattern(const cowa_pattern* pat, int Hkv, Pat* out) {
   const int H = pat->h_kv_global > 0 ? pat->h_kv_global : Hkv;
   if (pat->S < 0 || pat->T < pat->S || pat->L < 1 || pat->D < 1) return COWA_ERR_INVALID_ARG;
   if (H < 1 || H % pat->D != 0) return COWA_ERR_INVALID_ARG;
-  if (pat->kv_head_base < 0 || pat->kv_head_base + Hkv > H) return COWA_ERR_INVALID_ARG;
+  if (pat->kv_head_base < 0 || pat->kv_head_base > H - Hkv) return COWA_ERR_INVALID_ARG;  // no overflow
   out->S = pat->S; out->L = pat->L; out->T = pat->T; out->D = pat->D;
   out->G0 = pat->kv_head_base; out->H = H;
   return COWA_OK;

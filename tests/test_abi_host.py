@@ -155,6 +155,7 @@ def _fwd(pat, B=1, N=128, Hq=8, Hkv=4, d=128, q=None, lse=0x20000, ws=0x40000, w
     (dict(pat=cw.Pattern(64, 8, 1024, 4), ws_bytes=16), 4),
     (dict(pat=cw.Pattern(64, 8, 1024, 4), ws=0x40010), 4),  # workspace not 256-aligned
     (dict(pat=cw.Pattern(64, 8, 1024, 4, kv_head_base=2, h_kv_global=4)), 1),  # base + Hkv > H
+    (dict(pat=cw.Pattern(64, 8, 1024, 4, kv_head_base=2**31 - 2, h_kv_global=4)), 1),  # base + Hkv wraps
 ])
 def test_fwd_rejects_bad_arguments_before_launch(kwargs, status):
     assert _fwd(**kwargs) == status
