@@ -39,6 +39,8 @@ PLAN_CASES = [
     # N, Hkv, BM, BN, pattern
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 4)),       # tiny config
     (700, 2, 128, 128, cw.Pattern(16, 2**31 - 1, 700, 2)),   # window of INT_MAX (dense causal): no overflow
+    (700, 4, 128, 128, cw.Pattern(16, 50, 2**31 - 1, 4)),    # declared span of INT_MAX: intervals past N
+    (700, 2, 128, 128, cw.Pattern(2**31 - 1, 1, 2**31 - 1, 2)),  # sink of INT_MAX: every key a sink key
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 2)),       # duplicated D=2
     (1024, 4, 128, 128, cw.Pattern(64, 128, 1024, 1)),       # duplicated D=1
     (1000, 4, 128, 128, cw.Pattern(64, 128, 1000, 4)),       # ragged tail

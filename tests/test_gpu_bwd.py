@@ -80,6 +80,8 @@ def test_bwd_tiny_config(cuda_device, D):
     (1, 520, 4, 2, 64, cw.Pattern(4, 60, 4, 1)),             # SWA + sinks
     (1, 700, 8, 4, 128, cw.Pattern(32, 100, 500, 4)),        # N > T
     (1, 300, 2, 1, 128, cw.Pattern(7, 30, 300, 2, kv_head_base=1, h_kv_global=2)),  # TP rank
+    (1, 700, 8, 4, 128, cw.Pattern(16, 50, 2**31 - 1, 4)),   # declared span of INT_MAX: intervals past N
+    (1, 300, 4, 2, 64, cw.Pattern(2**31 - 1, 1, 2**31 - 1, 2)),  # sink of INT_MAX: dense causal
     (1, 256, 16, 2, 64, cw.Pattern(16, 64, 256, 2, softmax_scale=0.3)),  # group of 8
     (2, 1, 10, 2, 128, cw.Pattern(64, 128, 1024, 2)),       # N = 1: one key per row, dq = dk = 0
     (1, 300, 8, 4, 128, cw.Pattern(0, 1, 0, 4)),            # S = 0, L = 1, T = 0: each row sees only itself

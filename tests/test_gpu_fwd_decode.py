@@ -50,6 +50,8 @@ def test_fwd_tiny_config(cuda_device, D):
     (1, 700, 8, 4, 128, cw.Pattern(32, 100, 500, 4)),        # N > T
     (1, 300, 2, 1, 128, cw.Pattern(7, 30, 300, 2, kv_head_base=1, h_kv_global=2)),  # TP rank 1 of 2
     (1, 256, 16, 2, 64, cw.Pattern(16, 64, 256, 2, softmax_scale=0.3)),  # group of 8, explicit scale
+    (1, 700, 8, 4, 128, cw.Pattern(16, 50, 2**31 - 1, 4)),   # declared span of INT_MAX: intervals past N
+    (1, 300, 4, 2, 64, cw.Pattern(2**31 - 1, 1, 2**31 - 1, 2)),  # sink of INT_MAX: dense causal
 ])
 def test_fwd_edge_shapes(cuda_device, B, N, Hq, Hkv, d, pat):
     _check_fwd_full(B, N, Hq, Hkv, d, pat, cuda_device, extra=1)
