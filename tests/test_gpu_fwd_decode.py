@@ -246,6 +246,15 @@ def test_decode_small(cuda_device, d, Hq, Hkv):
     _check_decode(len(pos), Hq, Hkv, d, T_cap, pat, pos, cuda_device)
 
 
+@pytest.mark.parametrize("pat", [cw.Pattern(16, 50, 2**31 - 1, 4),         # intervals far past the cache
+                                 cw.Pattern(8, 2**31 - 1, 1024, 4),          # window of INT_MAX (dense)
+                                 cw.Pattern(2**31 - 1, 1, 2**31 - 1, 4)])    # every key a sink key
+def test_decode_extreme_patterns(cuda_device, pat):
+    """Pattern parameters at the int range's end: plans and chunking stay exact."""
+    pos = [0, 127, 640, 1023]
+    _check_decode(len(pos), 8, 4, 128, 1024, pat, pos, cuda_device)
+
+
 def test_decode_token_major_cache_and_duplicated_windows(cuda_device):
     pat = cw.Pattern(16, 100, 2000, 2)
     pos = [1999, 17, 1500, 100]
