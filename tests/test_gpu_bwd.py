@@ -44,6 +44,36 @@ def _check_full(B, N, Hq, Hkv, d, pat, device, extra=0):
     assert max(errs) <= GRAD_RTOL, errs
 
 
+def test_bwd_packed_qkv_layout(cuda_device):
+    """The fused-projection layout of training: q, k, v as views into one packed
+    [B, N, H_q + 2 H_kv, d] buffer, o and dO as views of wider buffers, and dq, dk, dv written
+    into the matching views of one packed gradient buffer (nothing else of it touched).  The
+    strided calls give the same bits as contiguous copies, and match the oracle."""
+    B, N, Hq, Hkv, d = 2, 600, 8, 2, 128
+    pat = cw.Pattern(32, 100, 600, 2)
+    W = Hq + 2 * Hkv
+    qkv64, qkv = host_and_device((B, N, W, d), "q", cuda_device, 13)
+    do64, dobuf = host_and_device((B, N, 2 * Hq, d), "do", cuda_device, 13)
+    q, k, v = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
+    do = dobuf[:, :, Hq:]
+    obuf = torch.zeros((B, N, 2 * Hq, d), dtype=torch.bfloat16, device=cuda_device)
+    o, lse = cw.cowa_fwd(q, k, v, pat, out=obuf[:, :, :Hq])
+    gbuf = torch.full((B, N, W + 2, d), 7.0, dtype=torch.bfloat16, device=cuda_device)  # 2 spare heads
+    dq, dk, dv = gbuf[:, :, :Hq], gbuf[:, :, Hq:Hq + Hkv], gbuf[:, :, Hq + Hkv:]
+    cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv)
+    qc, kc, vc, oc, doc = (x.contiguous() for x in (q, k, v, o, do))
+    ref = cw.cowa_bwd(qc, kc, vc, oc, lse, doc, pat)
+    torch.cuda.synchronize()
+    for got, want in zip((dq, dk, dv), ref):
+        assert torch.equal(got, want)
+    assert bool((gbuf[:, :, W:] == 7.0).all())
+    host = (qkv64[:, :, :Hq], qkv64[:, :, Hq:Hq + Hkv], qkv64[:, :, Hq + Hkv:], do64[:, :, Hq:])
+    op = oracle_pattern(pat)
+    want = orc.attention_bwd(*host, op)
+    errs = grad_errors((to64(dq), to64(dk), to64(dv)), want, grad_bounds(*host, op.sm_scale(d)))
+    assert max(errs) <= GRAD_RTOL, errs
+
+
 def test_window_of_int_max_equals_dense_causal(cuda_device):
     """A band of L = INT_MAX (a caller's "no window limit") is the dense-causal mode: forward and
     backward give the same bits as L = N, and the gradients match the oracle.  The band ends
