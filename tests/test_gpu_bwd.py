@@ -59,7 +59,7 @@ def test_bwd_packed_qkv_layout(cuda_device):
     obuf = torch.zeros((B, N, 2 * Hq, d), dtype=torch.bfloat16, device=cuda_device)
     o, lse = cw.cowa_fwd(q, k, v, pat, out=obuf[:, :, :Hq])
     gbuf = torch.full((B, N, W + 2, d), 7.0, dtype=torch.bfloat16, device=cuda_device)  # 2 spare heads
-    dq, dk, dv = gbuf[:, :, :Hq], gbuf[:, :, Hq:Hq + Hkv], gbuf[:, :, Hq + Hkv:]
+    dq, dk, dv = gbuf[:, :, :Hq], gbuf[:, :, Hq:Hq + Hkv], gbuf[:, :, Hq + Hkv:W]
     cw.cowa_bwd(q, k, v, o, lse, do, pat, dq=dq, dk=dk, dv=dv)
     qc, kc, vc, oc, doc = (x.contiguous() for x in (q, k, v, o, do))
     ref = cw.cowa_bwd(qc, kc, vc, oc, lse, doc, pat)
