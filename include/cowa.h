@@ -62,7 +62,10 @@ typedef enum {
   COWA_ERR_ALIGNMENT = 3,   /* pointer or stride not 16-byte aligned */
   COWA_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
   COWA_ERR_CUDA = 5,        /* CUDA runtime/driver error at launch */
-  COWA_ERR_TIMEOUT = 6      /* a device-side bounded wait ran out */
+  COWA_ERR_TIMEOUT = 6,     /* a device-side bounded wait ran out */
+  COWA_ERR_CHECK = 7        /* a device-side self-check of a COWA_DEBUG build failed (a planned
+                               tile or cache row outside the call's tensors); the access was
+                               skipped.  Release builds never report it. */
 } cowa_status;
 
 /* Window parameters of one attention layer.
@@ -297,7 +300,10 @@ cowa_status cowa_decode_noalloc_status(void* stream);
 
 /* ---- status --------------------------------------------------------------------------------
  * Synchronizes `stream`, reads and clears the device status word in `ws` (the workspace of an
- * earlier call), and returns COWA_OK or COWA_ERR_TIMEOUT (COWA_ERR_CUDA if the stream failed). */
+ * earlier call), and returns COWA_OK, COWA_ERR_TIMEOUT, or (debug builds) COWA_ERR_CHECK
+ * (COWA_ERR_CUDA if the stream failed).  A debug build records the first failed self-check in
+ * the two 32-bit words after the status word (a check code: 0x1nn forward, 0x2nn dK/dV, 0x3nn
+ * dQ, 0x4nn decode; and the offending tile index or cache row); they are cleared with it. */
 cowa_status cowa_workspace_status(void* ws, void* stream);
 const char* cowa_status_string(cowa_status s);
 

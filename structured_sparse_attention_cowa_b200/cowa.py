@@ -28,11 +28,13 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcowa.so")
+# COWA_DEBUG=1 selects the self-checking build (`python -m structured_sparse_attention_cowa_b200.build
+# --debug`); it computes the same bits and reports a failed check as COWA_ERR_CHECK
+LIB_PATH = os.path.join(_HERE, "libcowa_debug.so" if os.environ.get("COWA_DEBUG") == "1" else "libcowa.so")
 
 COWA_OK = 0
 _STATUS = {0: "COWA_OK", 1: "COWA_ERR_INVALID_ARG", 2: "COWA_ERR_UNSUPPORTED", 3: "COWA_ERR_ALIGNMENT",
-           4: "COWA_ERR_WORKSPACE", 5: "COWA_ERR_CUDA", 6: "COWA_ERR_TIMEOUT"}
+           4: "COWA_ERR_WORKSPACE", 5: "COWA_ERR_CUDA", 6: "COWA_ERR_TIMEOUT", 7: "COWA_ERR_CHECK"}
 
 BWD_PREPROCESS, BWD_DKDV, BWD_DQ = 1, 2, 4
 
@@ -79,8 +81,9 @@ def lib() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"libcowa.so not found at {LIB_PATH}; build it with "
-                           "`python -m structured_sparse_attention_cowa_b200.build`")
+        raise RuntimeError(f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}; build it with "
+                           "`python -m structured_sparse_attention_cowa_b200.build`"
+                           + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
     L = ctypes.CDLL(LIB_PATH)
     P, T, vp, i, sz = ctypes.POINTER(c_pattern), c_tensor, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.cowa_fwd_workspace_size.argtypes = [P, i, i, i, i, i]

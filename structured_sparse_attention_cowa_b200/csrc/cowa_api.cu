@@ -142,6 +142,7 @@ const char* cowa_status_string(cowa_status s) {
     case COWA_ERR_WORKSPACE: return "workspace too small, null or not 256-byte aligned";
     case COWA_ERR_CUDA: return "CUDA error";
     case COWA_ERR_TIMEOUT: return "a device-side bounded wait ran out";
+    case COWA_ERR_CHECK: return "a device-side self-check of the debug build failed";
   }
   return "unknown status";
 }
@@ -153,9 +154,10 @@ cowa_status cowa_workspace_status(void* ws, void* stream) {
   if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return COWA_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return COWA_ERR_CUDA;
   if (word != 0) {
-    if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return COWA_ERR_CUDA;
+    // clear the status word and the self-check record (words 1 and 2) for the next call
+    if (cudaMemsetAsync(ws, 0, 3 * sizeof(word), s) != cudaSuccess) return COWA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return COWA_ERR_CUDA;
-    return COWA_ERR_TIMEOUT;
+    return (word & 2u) ? COWA_ERR_CHECK : COWA_ERR_TIMEOUT;
   }
   return COWA_OK;
 }

@@ -173,16 +173,24 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
     if (lane == 0) {
       ptx::tma_prefetch_desc(&a.tm_q);
       ptx::tma_prefetch_desc(&a.tm_do);
-      ptx::mbar_arrive_expect_tx(&kv_full, 2 * Geo::kTileBytes);
-      for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sK + u * 16384, &a.tm_k, &kv_full, u * 64, row0 + s0, g, b);
-        ptx::tma_load_4d(sV + u * 16384, &a.tm_v, &kv_full, u * 64, row0 + s0, g, b);
+      // (debug builds) the key tile lies inside the sequence, the head and batch inside the call
+      const bool kv_ok = ptx::dbg_check(s0 >= 0 && s0 < N && g < a.Hkv && b < a.B, a.status, &abort_flag, 0x201, s0);
+      if (kv_ok) {
+        ptx::mbar_arrive_expect_tx(&kv_full, 2 * Geo::kTileBytes);
+        for (int u = 0; u < D / 64; ++u) {
+          ptx::tma_load_4d(sK + u * 16384, &a.tm_k, &kv_full, u * 64, row0 + s0, g, b);
+          ptx::tma_load_4d(sV + u * 16384, &a.tm_v, &kv_full, u * 64, row0 + s0, g, b);
+        }
       }
       int issued = 0;
-      for (int n = 0; n < nsteps; ++n) {
+      for (int n = 0; kv_ok && n < nsteps; ++n) {
         const int slot = n & 1;
         if (n >= 2 && !ptx::mbar_wait(&slot_empty[slot], ((n >> 1) - 1) & 1, &abort_flag, a.status)) break;
         const int i = i_lo + n / grp, h = g * grp + n % grp;
+        // (debug builds) the planned query tile lies inside the sequence and its statistics
+        if (!ptx::dbg_check(i >= 0 && i * kTile < N && h < a.Hq && (tile0 + i + 1) * kTile <= a.N_pad, a.status,
+                            &abort_flag, 0x202, i))
+          break;
         uint8_t* dst = sSlot + slot * Geo::kSlotKV;
         ptx::mbar_arrive_expect_tx(&slot_full[slot], Geo::kSlotKV);
         for (int u = 0; u < D / 64; ++u) {
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
         ptx::bulk_load(dst + 2 * Geo::kTileBytes + 512, a.delta + so, 512, &slot_full[slot]);
         issued = n + 1;
       }
-      ptx::mbar_wait(&kv_full, 0, nullptr, a.status);
+      if (kv_ok) ptx::mbar_wait(&kv_full, 0, nullptr, a.status);
       for (int n = (issued > 2 ? issued - 2 : 0); n < issued; ++n)
         ptx::mbar_wait(&slot_full[n & 1], (n >> 1) & 1, nullptr, a.status);
     }
@@ -463,17 +471,23 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
     if (lane == 0) {
       ptx::tma_prefetch_desc(&a.tm_k);
       ptx::tma_prefetch_desc(&a.tm_v);
-      ptx::mbar_arrive_expect_tx(&q_full, 2 * Geo::kTileBytes);
-      for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + t0, h, b);
-        ptx::tma_load_4d(sDO + u * 16384, &a.tm_do, &q_full, u * 64, row0 + t0, h, b);
+      // (debug builds) the query tile lies inside the sequence, the head and batch inside the call
+      const bool q_ok = ptx::dbg_check(t0 >= 0 && t0 < N && h < a.Hq && b < a.B, a.status, &abort_flag, 0x301, t0);
+      if (q_ok) {
+        ptx::mbar_arrive_expect_tx(&q_full, 2 * Geo::kTileBytes);
+        for (int u = 0; u < D / 64; ++u) {
+          ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + t0, h, b);
+          ptx::tma_load_4d(sDO + u * 16384, &a.tm_do, &q_full, u * 64, row0 + t0, h, b);
+        }
       }
       TileCursor cur;
       cur.init(T);
       int issued = 0;
-      for (int n = 0; n < ntiles; ++n, cur.next(T)) {
+      for (int n = 0; q_ok && n < ntiles; ++n, cur.next(T)) {
         const int ks = n % KS, vs = n % VS;
         if (n >= KS && !ptx::mbar_wait(&k_empty[ks], ((n / KS) - 1) & 1, &abort_flag, a.status)) break;
+        // (debug builds) every planned KV tile lies inside the sequence
+        if (!ptx::dbg_check(cur.j >= 0 && cur.j * kTile < N, a.status, &abort_flag, 0x302, cur.j)) break;
         ptx::mbar_arrive_expect_tx(&k_full[ks], Geo::kTileBytes);
         for (int u = 0; u < D / 64; ++u)
           ptx::tma_load_4d(sK + ks * Geo::kTileBytes + u * 16384, &a.tm_k, &k_full[ks], u * 64, row0 + cur.j * kTile,
@@ -489,7 +503,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dq_kernel(const __gr
         issued = n + 1;
       }
       // drain: every copy issued must have landed before the CTA exits
-      ptx::mbar_wait(&q_full, 0, nullptr, a.status);
+      if (q_ok) ptx::mbar_wait(&q_full, 0, nullptr, a.status);
       const int nk = issued < 0 ? -issued : issued, nv = issued < 0 ? -issued - 1 : issued;
       for (int n = (nk > KS ? nk - KS : 0); n < nk; ++n) ptx::mbar_wait(&k_full[n % KS], (n / KS) & 1, nullptr, a.status);
       for (int n = (nv > VS ? nv - VS : 0); n < nv; ++n) ptx::mbar_wait(&v_full[n % VS], (n / VS) & 1, nullptr, a.status);

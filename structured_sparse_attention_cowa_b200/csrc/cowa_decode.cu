@@ -203,8 +203,12 @@ __device__ __forceinline__ void decode_split_body(const DecodeArgs& a) {
         if (st >= kStages && !ptx::mbar_wait(&empty_bar[s], ph ^ 1, &abort_flag, a.status)) break;
         uint8_t* ks = smem + s * Geo::kStageBytes;
         uint8_t* vs = ks + Geo::kTileBytes;
-        ptx::mbar_arrive_expect_tx(&full_bar[s], Geo::kStageBytes);
         const int row = cache_row(p_base + st * kSubTok);
+        // (debug builds) the sub-tile starts inside the cache (a compacted block ends inside it too)
+        if (!ptx::dbg_check(row >= 0 && (a.compact ? row + kSubTok <= a.cg.rows : row < a.T_cap) && b < a.B,
+                            a.status, &abort_flag, 0x401, row))
+          break;
+        ptx::mbar_arrive_expect_tx(&full_bar[s], Geo::kStageBytes);
 #pragma unroll
         for (int u = 0; u < Geo::kUnits; ++u) {
           ptx::tma_load_4d(ks + u * kBoxBytes, &a.tm_k, &full_bar[s], u * Geo::kBoxElems, row, g, b);

@@ -152,17 +152,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
       ptx::tma_prefetch_desc(&a.tm_q);
       ptx::tma_prefetch_desc(&a.tm_k);
       ptx::tma_prefetch_desc(&a.tm_v);
-      ptx::mbar_arrive_expect_tx(&q_full, (has1 ? 2 : 1) * Geo::kQBytes);
-      for (int u = 0; u < D / 64; ++u) {
-        ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0, b);
-        if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0 + 1, b);
+      // (debug builds) the work item addresses rows and heads of the call
+      const bool q_ok = ptx::dbg_check(i >= 0 && i * kBM < Nq && h0 + (has1 ? 1 : 0) < a.Hq && b < a.B, a.status,
+                                       &abort_flag, 0x101, i);
+      if (q_ok) {
+        ptx::mbar_arrive_expect_tx(&q_full, (has1 ? 2 : 1) * Geo::kQBytes);
+        for (int u = 0; u < D / 64; ++u) {
+          ptx::tma_load_4d(sQ + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0, b);
+          if (has1) ptx::tma_load_4d(sQ + Geo::kQBytes + u * 16384, &a.tm_q, &q_full, u * 64, row0 + i * kBM, h0 + 1, b);
+        }
       }
       TileCursor cur;
       cur.init(T);
       int issued = 0;
-      for (int idx = 0; idx < 2 * ntiles; ++idx) {
+      for (int idx = 0; q_ok && idx < 2 * ntiles; ++idx) {
         const int s = idx % Geo::kRing;
         if (idx >= Geo::kRing && !ptx::mbar_wait(&kv_empty[s], ((idx / Geo::kRing) - 1) & 1, &abort_flag, a.status)) break;
+        // (debug builds) every planned KV tile lies inside the keys of the call
+        if (!ptx::dbg_check(cur.j >= 0 && cur.j * kBN < Nk, a.status, &abort_flag, 0x102, cur.j)) break;
         const bool is_v = idx & 1;
         uint8_t* dst = sRing + s * Geo::kKVBytes;
         ptx::mbar_arrive_expect_tx(&kv_full[s], Geo::kKVBytes);
@@ -172,7 +179,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) cowa_fwd_kernel(const __grid_c
         issued = idx + 1;
       }
       // drain: no copy may still be landing in shared memory when the CTA exits
-      ptx::mbar_wait(&q_full, 0, nullptr, a.status);
+      if (q_ok) ptx::mbar_wait(&q_full, 0, nullptr, a.status);
       for (int idx = (issued > Geo::kRing ? issued - Geo::kRing : 0); idx < issued; ++idx)
         ptx::mbar_wait(&kv_full[idx % Geo::kRing], (idx / Geo::kRing) & 1, nullptr, a.status);
     }

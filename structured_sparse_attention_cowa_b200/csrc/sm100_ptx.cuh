@@ -110,8 +110,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Status codes written to the workspace status word when a wait gives up.
-enum : uint32_t { kStatusTimeout = 1u };
+// Status bits of the workspace status word (word 0 of the workspace header): a bounded wait
+// gave up, or (COWA_DEBUG builds) a self-check failed.
+enum : uint32_t { kStatusTimeout = 1u, kStatusCheck = 2u };
 
 // Bounded wait on the phase with the given parity.  Returns false if the
 // wait ran out (about `limit_ns` of wall time) or if another thread of the CTA
@@ -137,6 +138,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
+}
+
+// Self-check of a COWA_DEBUG build (release builds compile it to `true`): when `cond` fails it
+// records `code` and `value` in header words 1 and 2 (the first failure of the launch wins), sets
+// kStatusCheck, raises the CTA's abort flag and returns false, and the caller skips the access
+// that the check guards.  It never traps: the other warps leave through their bounded waits.
+__device__ __forceinline__ bool dbg_check(bool cond, uint32_t* status, volatile int* abort, uint32_t code,
+                                          int value) {
+#if defined(COWA_DEBUG) && COWA_DEBUG
+  if (!cond) {
+    if (status) {
+      if (atomicCAS(status + 1, 0u, code) == 0u) status[2] = (uint32_t)value;
+      atomicOr(status, kStatusCheck);
+    }
+    if (abort) *abort = 1;
+    return false;
+  }
+#else
+  (void)cond; (void)status; (void)abort; (void)code; (void)value;
+#endif
+  return true;
 }
 
 // Warp-uniform variant: every lane waits, and the warp proceeds only if all lanes saw the

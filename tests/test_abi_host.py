@@ -30,6 +30,16 @@ def test_library_exports_every_declared_symbol():
     assert L.cowa_version() >= 1
 
 
+def test_debug_library_builds_and_exports_every_declared_symbol():
+    """The self-checking build (COWA_DEBUG=1, libcowa_debug.so) is the same ABI."""
+    from structured_sparse_attention_cowa_b200 import build as cbuild
+
+    L = ctypes.CDLL(cbuild.build(debug=True))
+    for n in _declared_functions():
+        assert hasattr(L, n), n
+    assert L.cowa_status_string(7) != 0
+
+
 def _oracle_pattern(p: cw.Pattern):
     return orc.Pattern(S=p.S, L=p.L, T=p.T, D=p.D, kv_head_base=p.kv_head_base,
                        h_kv_global=p.h_kv_global or None)
