@@ -496,7 +496,7 @@ cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H
 size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d) {
   Pat p;
   if (check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(B, N, Hq, Hkv, d) != COWA_OK) return 0;
-  return kWsHeader + bwd_workspace_bytes(B, N, Hq, Hkv, d);
+  return kWsHeader + bwd_workspace_bytes(p, B, N, Hq, Hkv, d);
 }
 
 cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int Hq, int Hkv, int d, cowa_tensor q, cowa_tensor k,
@@ -534,6 +534,18 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int H
   a.N_pad = (N + 127) / 128 * 128;
   a.delta = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader);
   a.lse2 = a.delta + (size_t)B * Hq * a.N_pad;
+  {
+    // long dK/dV key tiles split by query range: chunk table and fp32 partials after the statistics
+    const KvSplit sp = kv_split_plan(p, B, N, Hq, Hkv);
+    if (sp.chunk > 0) {
+      if (sp.n_entries > 0x7fffffffLL) return COWA_ERR_UNSUPPORTED;
+      char* base = reinterpret_cast<char*>(ws) + kWsHeader + align_up(2 * (size_t)B * Hq * a.N_pad * sizeof(float), 256);
+      a.kv_chunk = sp.chunk;
+      a.n_split = (int)sp.n_entries;
+      a.kv_tab = reinterpret_cast<int4*>(base);
+      a.kv_part = reinterpret_cast<float*>(base + align_up((size_t)sp.n_entries * sizeof(int4), 256));
+    }
+  }
   a.scale = scale_of(pat, d);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   if (!make_tmap_bf16(&a.tm_q, q.ptr, d, N, Hq, B, q.stride_t, q.stride_h, q.stride_b, 128) ||

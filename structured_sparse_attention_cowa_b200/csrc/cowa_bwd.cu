@@ -123,10 +123,18 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = a.Hq / a.Hkv;
-  // lowest key tiles first: their query ranges (sink, early intervals) are the longest
-  int j = blockIdx.x / (a.Hkv * a.B);
-  const int rem = blockIdx.x % (a.Hkv * a.B);
-  const int g = rem % a.Hkv, b = rem / a.Hkv;
+  // the chunks of split key tiles first (each about the mean work of an SM), then every key tile,
+  // lowest first: their query ranges (sink, early intervals) are the longest
+  int j, g, b, kc = -1;  // kc >= 0: chunk kc of a split key tile
+  if ((int)blockIdx.x < a.n_split) {
+    const int4 e = a.kv_tab[blockIdx.x];
+    j = e.x; g = e.y; b = e.z; kc = e.w;
+  } else {
+    const int x = (int)blockIdx.x - a.n_split;
+    j = x / (a.Hkv * a.B);
+    const int rem = x % (a.Hkv * a.B);
+    g = rem % a.Hkv; b = rem / a.Hkv;
+  }
   // the rows of this CTA's sequence: [row0, row0 + N) of the token axis; statistics tiles from tile0
   int row0 = 0, N = a.N, tile0 = 0;
   if (a.varlen) {
@@ -140,7 +148,12 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
   const int s0 = j * kTile, s1 = imin(N, s0 + kTile);
   const Range iv = interval_of(a.pat, g);
   const Range rows = bwd_row_range(a.pat, iv, s0, s1, N);
-  const int i_lo = rows.lo / kTile, i_hi = (rows.hi + kTile - 1) / kTile;
+  int i_lo = rows.lo / kTile, i_hi = (rows.hi + kTile - 1) / kTile;
+  if (a.kv_chunk > 0 && i_hi - i_lo > a.kv_chunk) {
+    if (kc < 0) return;  // a split tile: its chunk CTAs do the work (before any barrier or TMEM use)
+    i_lo += kc * a.kv_chunk;
+    i_hi = imin(i_hi, i_lo + a.kv_chunk);
+  }
   const int nsteps = (i_hi - i_lo) * grp;
 
   uint8_t* sK = smem;
@@ -364,7 +377,20 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
         ptx::tmem_ld32(lane_base + Geo::kColAcc + D + part * HC + c * 32, dkv + c * 32);
       }
       ptx::tmem_wait_ld();
-      if (s < N) {
+      if (kc >= 0) {
+        // a chunk of a split tile: fp32 partials [dV | dK][128 key rows][D], dK not yet scaled
+        float* pv = a.kv_part + (size_t)blockIdx.x * 2 * kTile * D + (size_t)r * D + part * HC;
+        float* pk = pv + (size_t)kTile * D;
+#pragma unroll
+        for (int c4 = 0; c4 < HC / 4; ++c4) {
+          reinterpret_cast<float4*>(pv)[c4] =
+              make_float4(__uint_as_float(dvv[4 * c4]), __uint_as_float(dvv[4 * c4 + 1]),
+                          __uint_as_float(dvv[4 * c4 + 2]), __uint_as_float(dvv[4 * c4 + 3]));
+          reinterpret_cast<float4*>(pk)[c4] =
+              make_float4(__uint_as_float(dkv[4 * c4]), __uint_as_float(dkv[4 * c4 + 1]),
+                          __uint_as_float(dkv[4 * c4 + 2]), __uint_as_float(dkv[4 * c4 + 3]));
+        }
+      } else if (s < N) {
         __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + ((int64_t)row0 + s) * a.dv_st +
                              g * a.dv_sh + part * HC;
         __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + ((int64_t)row0 + s) * a.dk_st +
@@ -685,6 +711,80 @@ constexpr int kDqParts = D == 128 ? COWA_DQ_PARTS : 2;
 template <int D>
 constexpr int kDkdvParts = D == 128 ? COWA_DKDV_PARTS : 2;
 
+// ------------------------------------------------------------------------------ split key tiles
+// Query tiles of key tile j for local KV head g (the dK/dV kernel's range).
+__host__ __device__ __forceinline__ int kv_range_tiles(const Pat& p, Range iv, int j, int N) {
+  const int s0 = j * kTile, s1 = imin(N, s0 + kTile);
+  const Range r = bwd_row_range(p, iv, s0, s1, N);
+  return (r.hi + kTile - 1) / kTile - r.lo / kTile;
+}
+
+// The chunk table of a split call (one block): every key tile (g-major, then j) whose range
+// exceeds `chunk` query tiles contributes ceil(range / chunk) consecutive entries {j, g, b, k},
+// batch element by batch element (entries of b at b * per_b).
+__global__ void __launch_bounds__(256) kv_split_table_kernel(Pat p, int N, int B, int Hkv, int chunk, int4* tab) {
+  __shared__ int offs[256];
+  __shared__ int per_b;
+  const int nq = (N + kTile - 1) / kTile, pairs = Hkv * nq, t = threadIdx.x;
+  const int per = (pairs + 255) / 256;
+  const int lo = imin(pairs, t * per), hi = imin(pairs, lo + per);
+  int cnt = 0;
+  for (int q = lo; q < hi; ++q) {
+    const int g = q / nq, j = q % nq;
+    const int n = kv_range_tiles(p, interval_of(p, g), j, N);
+    if (n > chunk) cnt += (n + chunk - 1) / chunk;
+  }
+  offs[t] = cnt;
+  __syncthreads();
+  if (t == 0) {  // exclusive scan of 256 counts, in order
+    int acc = 0;
+    for (int i = 0; i < 256; ++i) { const int v = offs[i]; offs[i] = acc; acc += v; }
+    per_b = acc;
+  }
+  __syncthreads();
+  int e = offs[t];
+  for (int q = lo; q < hi; ++q) {
+    const int g = q / nq, j = q % nq;
+    const int n = kv_range_tiles(p, interval_of(p, g), j, N);
+    if (n <= chunk) continue;
+    for (int k = 0; k < (n + chunk - 1) / chunk; ++k, ++e)
+      for (int bb = 0; bb < B; ++bb) tab[(size_t)bb * per_b + e] = make_int4(j, g, bb, k);
+  }
+}
+
+// dk, dv of the split key tiles: the chunks' fp32 partials summed in chunk order (one block per
+// tile, run by the block of its first chunk), dk scaled, rounded to bf16.
+template <int D>
+__global__ void __launch_bounds__(256) kv_split_reduce_kernel(const __grid_constant__ BwdArgs a) {
+  const int e0 = blockIdx.x;
+  const int4 t = a.kv_tab[e0];
+  if (t.w != 0) return;
+  const int j = t.x, g = t.y, b = t.z;
+  int n = 1;  // the tile's chunks are consecutive entries
+  while (e0 + n < a.n_split && a.kv_tab[e0 + n].w == n) ++n;
+  const int s0 = j * kTile;
+  for (int idx = threadIdx.x; idx < kTile * D / 4; idx += blockDim.x) {
+    const int r = idx / (D / 4), c4 = idx % (D / 4);
+    float4 sv = make_float4(0.f, 0.f, 0.f, 0.f), sk = sv;
+    for (int c = 0; c < n; ++c) {
+      const float* pp = a.kv_part + (size_t)(e0 + c) * 2 * kTile * D + (size_t)r * D;
+      const float4 v = reinterpret_cast<const float4*>(pp)[c4];
+      const float4 k = reinterpret_cast<const float4*>(pp + (size_t)kTile * D)[c4];
+      sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
+      sk.x += k.x; sk.y += k.y; sk.z += k.z; sk.w += k.w;
+    }
+    if (s0 + r < a.N) {
+      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + (int64_t)(s0 + r) * a.dv_st +
+                           g * a.dv_sh + c4 * 4;
+      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + (int64_t)(s0 + r) * a.dk_st +
+                           g * a.dk_sh + c4 * 4;
+      *reinterpret_cast<uint2*>(dvr) = make_uint2(ptx::pack_bf16(sv.x, sv.y), ptx::pack_bf16(sv.z, sv.w));
+      *reinterpret_cast<uint2*>(dkr) = make_uint2(ptx::pack_bf16(sk.x * a.scale, sk.y * a.scale),
+                                                  ptx::pack_bf16(sk.z * a.scale, sk.w * a.scale));
+    }
+  }
+}
+
 template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
   using Geo = BwdGeom<D>;
@@ -699,10 +799,18 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
     auto kdkdv = bwd_dkdv_kernel<D, NPK>;
     if ((e = cudaFuncSetAttribute(kdkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmemKV)) != cudaSuccess)
       return e;
-    const long long n_kv = (long long)nq * a.Hkv * a.B;
+    const long long n_kv = (long long)nq * a.Hkv * a.B + a.n_split;
     if (n_kv > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (a.n_split > 0) {
+      kv_split_table_kernel<<<1, 256, 0, s>>>(a.pat, a.N, a.B, a.Hkv, a.kv_chunk, a.kv_tab);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     kdkdv<<<(unsigned)n_kv, (4 * NPK + 2) * 32, Geo::kSmemKV, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.n_split > 0) {
+      kv_split_reduce_kernel<D><<<a.n_split, 256, 0, s>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
   }
   if (stages & COWA_BWD_DQ) {
     constexpr int NP = kDqParts<D>;
@@ -719,10 +827,50 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
 
 }  // namespace
 
-size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d) {
-  (void)Hkv; (void)d;
+// Split plan of a call (see BwdArgs).  A key tile whose query range is longer than the work an
+// SM averages over the launch would finish last whatever the order (a sink key tile walks every
+// query tile of every head of its group): with few KV heads per call (KV-head tensor
+// parallelism, layers with one or two KV heads) that one CTA sets the kernel's time.  Such
+// ranges are cut into chunks of about that mean work; calls whose longest range is within it
+// (the 8-head layers, where the other heads' tiles fill the SMs) are not split.
+KvSplit kv_split_plan(const Pat& p, int B, int N, int Hq, int Hkv) {
+  constexpr long long kSms = 148;  // B200
+  KvSplit sp{0, 0};
+  const int nq = (N + kTile - 1) / kTile, grp = Hq / Hkv;
+  long long total = 0;
+  int longest = 0;
+  for (int g = 0; g < Hkv; ++g) {
+    const Range iv = interval_of(p, g);
+    for (int j = 0; j < nq; ++j) {
+      const int n = kv_range_tiles(p, iv, j, N);
+      total += n;
+      longest = imax(longest, n);
+    }
+  }
+  // query tiles per SM over the launch, each costing grp heads x 2 sub-steps alike
+  const long long per_sm = total * B / kSms;
+  const int chunk = (int)(per_sm > 8 ? per_sm : 8);
+  if (longest <= chunk) return sp;
+  sp.chunk = chunk;
+  for (int g = 0; g < Hkv; ++g) {
+    const Range iv = interval_of(p, g);
+    for (int j = 0; j < nq; ++j) {
+      const int n = kv_range_tiles(p, iv, j, N);
+      if (n > chunk) sp.n_entries += (n + chunk - 1) / chunk;
+    }
+  }
+  sp.n_entries *= B;
+  (void)grp;
+  return sp;
+}
+
+size_t bwd_workspace_bytes(const Pat& p, int B, int N, int Hq, int Hkv, int d) {
   const size_t n_pad = (size_t)(N + kTile - 1) / kTile * kTile;
-  return align_up(2 * (size_t)B * Hq * n_pad * sizeof(float), 256);
+  size_t bytes = align_up(2 * (size_t)B * Hq * n_pad * sizeof(float), 256);
+  const KvSplit sp = kv_split_plan(p, B, N, Hq, Hkv);
+  if (sp.chunk > 0)
+    bytes += align_up((size_t)sp.n_entries * sizeof(int4), 256) + (size_t)sp.n_entries * 2 * kTile * d * sizeof(float);
+  return bytes;
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, int stages, cudaStream_t s) {

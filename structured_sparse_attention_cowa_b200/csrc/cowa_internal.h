@@ -115,9 +115,23 @@ struct BwdArgs {
   uint32_t* status;
   float scale;       // softmax scale
   float scale_log2;  // softmax scale * log2(e)
+  // Query-range split of long dK/dV key tiles (kv_chunk > 0; see kv_split_plan): the grid
+  // starts with n_split CTAs, one per chunk kv_tab[e] = {key tile, KV head, batch, chunk} of
+  // kv_chunk query tiles; each writes fp32 partial dV, dK ([2][128][d]) to kv_part + e*2*128*d,
+  // and a reduction kernel sums a tile's chunks in chunk order.  The unsplit CTA of such a tile
+  // leaves at once.  Packed batches do not split (kv_chunk = 0).
+  int kv_chunk, n_split;
+  int4* kv_tab;
+  float* kv_part;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
 };
-size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int d);
+struct KvSplit {
+  int chunk;             // query tiles per chunk; 0: no key tile is split
+  long long n_entries;   // chunks over all split key tiles and batch elements
+};
+KvSplit kv_split_plan(const Pat& p, int B, int N, int Hq, int Hkv);
+// workspace after the header: Delta, lse2, then (split calls) the chunk table and partials
+size_t bwd_workspace_bytes(const Pat& p, int B, int N, int Hq, int Hkv, int d);
 cudaError_t launch_bwd(const BwdArgs& a, int stages, cudaStream_t s);
 
 // ---- bounded-wait probe ----

@@ -258,6 +258,24 @@ def test_compact_layout_holds_every_visible_key_at_every_position(pat, Hkv):
                 assert blk[2] <= blk[0] and blk[1] <= blk[3], (g, t, s_, blk)
 
 
+def test_bwd_workspace_holds_the_split_of_long_key_tiles():
+    """The backward splits long dK/dV key tiles only when a call has few KV heads: the 8-head 32K
+    layer needs only the row statistics, one of its KV heads alone (a rank of KV-head tensor
+    parallelism) also the chunk table and fp32 partials."""
+    L = cw.lib()
+
+    def ws(pat, B, N, Hq, Hkv):
+        return L.cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, 128)
+
+    stats = 256 + 2 * 40 * 32768 * 4
+    assert ws(cw.Pattern(128, 2048, 32768, 8), 1, 32768, 40, 8) == stats
+    one = ws(cw.Pattern(128, 2048, 32768, 8, kv_head_base=0, h_kv_global=8), 1, 32768, 5, 1)
+    # head 0: the sink tile and the 32 tiles of its interval, in chunks of 78 query tiles
+    assert one == 256 + 2 * 5 * 32768 * 4 + (121 * 16 + 255) // 256 * 256 + 121 * 2 * 128 * 128 * 4
+    last = ws(cw.Pattern(128, 2048, 32768, 8, kv_head_base=7, h_kv_global=8), 1, 32768, 5, 1)
+    assert last == 256 + 2 * 5 * 32768 * 4 + 256 + 13 * 2 * 128 * 128 * 4
+
+
 def test_compact_entry_points_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(20, 100, 2000, 2).c()

@@ -44,6 +44,39 @@ def _check_full(B, N, Hq, Hkv, d, pat, device, extra=0):
     assert max(errs) <= GRAD_RTOL, errs
 
 
+def _unsplit_ws_bytes(B, N, Hq):
+    n_pad = (N + 127) // 128 * 128
+    return 256 + (2 * B * Hq * n_pad * 4 + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,pat", [
+    (1, 4096, 4, 1, 128, cw.Pattern(64, 256, 4096, 1)),     # one KV head: every key tile long
+    (2, 3000, 2, 1, 64, cw.Pattern(16, 64, 3000, 1)),       # two sequences, ragged, d = 64
+    (1, 4096, 4, 2, 128, cw.Pattern(32, 128, 4096, 2)),     # two KV heads: sink and interval tiles long
+])
+def test_bwd_split_key_tiles(cuda_device, B, N, Hq, Hkv, d, pat):
+    """Calls with few KV heads cut the query range of their long key tiles into chunks run by
+    CTAs of their own (fp32 partials summed in chunk order); the gradients match the oracle and
+    two calls give the same bits."""
+    import ctypes
+    ws_bytes = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+    assert ws_bytes > _unsplit_ws_bytes(B, N, Hq)  # the plan splits this call
+    host, dev = _inputs(B, N, Hq, Hkv, d, cuda_device, extra=17)
+    q, k, v, do = dev
+    o, lse = cw.cowa_fwd(q, k, v, pat)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=cuda_device)
+    g1 = cw.cowa_bwd(q, k, v, o, lse, do, pat, workspace=ws)
+    g2 = cw.cowa_bwd(q, k, v, o, lse, do, pat, workspace=ws)
+    torch.cuda.synchronize()
+    assert cw.workspace_status(ws) == 0
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
+    op = oracle_pattern(pat)
+    want = orc.attention_bwd(*host, op)
+    errs = grad_errors(tuple(to64(x) for x in g1), want, grad_bounds(*host, op.sm_scale(d)))
+    assert max(errs) <= GRAD_RTOL, errs
+
+
 def test_bwd_packed_qkv_layout(cuda_device):
     """The fused-projection layout of training: q, k, v as views into one packed
     [B, N, H_q + 2 H_kv, d] buffer, o and dO as views of wider buffers, and dq, dk, dv written
