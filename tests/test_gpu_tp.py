@@ -13,6 +13,7 @@ import torch
 from oracle import cowa_oracle as orc
 from structured_sparse_attention_cowa_b200 import cowa as cw
 from structured_sparse_attention_cowa_b200 import shard
+from structured_sparse_attention_cowa_b200 import synth
 from tests.gpu_helpers import GRAD_RTOL, LSE_ATOL, O_ATOL, grad_bounds, grad_errors, host_and_device, oracle_pattern, to64
 
 pytestmark = pytest.mark.gpu
@@ -71,3 +72,39 @@ def test_tp_decode_runs_reproduce_the_layer(cuda_device):
             torch.cuda.synchronize()
             assert np.abs(to64(o) - want_o[:, qh.start:qh.stop]).max() <= O_ATOL, (r, run)
             assert np.abs(lse.cpu().numpy() - want_l[:, qh.start:qh.stop]).max() <= LSE_ATOL, (r, run)
+
+
+@pytest.mark.parametrize("g", [0, 7])
+def test_tp_rank_of_one_kv_head_at_32k_matches_the_layer(cuda_device, g):
+    """A rank holding one KV head of the 32K layer (H_q = 40, H_kv = 8, S = 128, L = 2048): its
+    backward call splits the long key tiles (head 0: 121 chunks, head 7: 13) and reproduces
+    that head of the unsplit 8-head call.  dq is the same kernel on the same rows (equal bits);
+    dk, dv differ only by the fp32 order of the chunks' partial sums (bf16 rounding)."""
+    import ctypes
+
+    B, N, Hq, Hkv, d = 1, 32768, 40, 8, 128
+    grp = Hq // Hkv
+    q, k, v, do = (synth.cuda_normal_bf16(s, synth.seed_of(n, 41), cuda_device)
+                   for s, n in (((B, N, Hq, d), "q"), ((B, N, Hkv, d), "k"), ((B, N, Hkv, d), "v"),
+                                ((B, N, Hq, d), "do")))
+    layer = cw.Pattern(128, 2048, 32768, 8)
+    o, lse = cw.cowa_fwd(q, k, v, layer)
+    dq, dk, dv = cw.cowa_bwd(q, k, v, o, lse, do, layer)
+    one = cw.Pattern(128, 2048, 32768, 8, kv_head_base=g, h_kv_global=8)
+    hq = slice(g * grp, (g + 1) * grp)
+    qg, kg, vg, dog = (x.contiguous() for x in (q[:, :, hq], k[:, :, g:g + 1], v[:, :, g:g + 1], do[:, :, hq]))
+    og, lseg = cw.cowa_fwd(qg, kg, vg, one)
+    assert torch.equal(og, o[:, :, hq]) and torch.equal(lseg, lse[:, hq])
+    L = cw.lib()
+    n_ws = L.cowa_bwd_workspace_size(ctypes.byref(one.c()), B, N, grp, 1, d)
+    assert n_ws > 256 + 2 * grp * N * 4  # the call splits its long key tiles
+    ws = torch.zeros(n_ws, dtype=torch.uint8, device=cuda_device)
+    dqg, dkg, dvg = cw.cowa_bwd(qg, kg, vg, og, lseg, dog, one, workspace=ws)
+    torch.cuda.synchronize()
+    assert cw.workspace_status(ws) == 0
+    assert torch.equal(dqg, dq[:, :, hq])
+    for got, want in ((dkg, dk[:, :, g:g + 1]), (dvg, dv[:, :, g:g + 1])):
+        a, b = got.float(), want.float()
+        rel = float((a - b).norm() / b.norm())
+        assert rel <= 2e-3, rel
+        assert float((a == b).float().mean()) >= 0.9  # most elements round to the same bf16
