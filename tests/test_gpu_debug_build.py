@@ -3,9 +3,9 @@
 In that build every kernel checks each planned tile and cache row against the call's tensors
 before its TMA load (a failed check reports COWA_ERR_CHECK through the workspace status and
 skips the load; nothing traps).  On the awkward shapes below (ragged tails, GQA groups of 1 and
-5, N > T, dense causal, d = 64, a packed batch with empty and length-1 sequences, a chunk of
-queries against a decode cache, full and compacted caches in bf16 and E4M3) no check fails and
-every output equals the release build's bit for bit."""
+5, N > T, dense causal, d = 64, one KV head (split key tiles), a packed batch with empty and
+length-1 sequences, a chunk of queries against a decode cache, full and compacted caches in bf16
+and E4M3) no check fails and every output equals the release build's bit for bit."""
 
 import pytest
 import torch
@@ -58,6 +58,7 @@ def _rand(shape, name, extra, device):
     (1, 700, 8, 4, 128, cw.Pattern(32, 100, 500, 4)),         # N > T
     (1, 640, 8, 2, 128, cw.Pattern(16, 640, 640, 2)),         # dense causal
     (1, 300, 8, 4, 64, cw.Pattern(8, 32, 300, 2)),            # d = 64, duplicated windows
+    (1, 4096, 4, 1, 128, cw.Pattern(64, 256, 4096, 1)),       # one KV head: long key tiles split
 ])
 def test_debug_build_fwd_bwd(libs, cuda_device, B, N, Hq, Hkv, d, pat):
     q, k, v, do = (_rand(s, n, 21, cuda_device) for s, n in (((B, N, Hq, d), "q"), ((B, N, Hkv, d), "k"),
