@@ -560,6 +560,22 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int Hq, int H
 namespace {
 // 128 x the tile bound of a packed batch: every sequence's statistics start at its own tile
 long long packed_rows_pad(int total, int n_seq) { return packed_tiles_bound(total, n_seq) * 128; }
+
+// The key-tile split of a packed batch is planned as for one sequence of all `total` rows (the
+// longest ranges a batch of that size can have); the device fills a table of `cap` slots.
+int varlen_split_cap(const Pat& p, int total, int Hq, int Hkv, int* chunk) {
+  const KvSplit sp = kv_split_plan(p, 1, total, Hq, Hkv);
+  *chunk = sp.chunk;
+  if (sp.chunk == 0) return 0;
+  const long long cap = 2 * sp.n_entries + 64;
+  return cap > 0x7fffffffLL ? -1 : (int)cap;
+}
+
+size_t varlen_split_bytes(int cap, int Hkv, long long rows, int d) {
+  if (cap <= 0) return 0;
+  return align_up((size_t)Hkv * (size_t)(rows / 128) * sizeof(int32_t), 256) + align_up((size_t)cap * sizeof(int4), 256) +
+         (size_t)cap * 2 * 128 * d * sizeof(float);
+}
 }  // namespace
 
 size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d) {
@@ -567,7 +583,11 @@ size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int to
   if (n_seq < 1 || check_pattern(pat, Hkv, &p) != COWA_OK || check_heads(1, total, Hq, Hkv, d) != COWA_OK) return 0;
   const long long rows = packed_rows_pad(total, n_seq);
   if (rows > 0x7fffffffLL) return 0;
-  return kWsHeader + seq_table_bytes(n_seq) + align_up(2 * (size_t)Hq * (size_t)rows * sizeof(float), 256);
+  int chunk;
+  const int cap = varlen_split_cap(p, total, Hq, Hkv, &chunk);
+  if (cap < 0) return 0;
+  return kWsHeader + seq_table_bytes(n_seq) + align_up(2 * (size_t)Hq * (size_t)rows * sizeof(float), 256) +
+         varlen_split_bytes(cap, Hkv, rows, d);
 }
 
 cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, int total, int Hq, int Hkv, int d,
@@ -602,6 +622,22 @@ cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H
   a.N_pad = (int)packed_rows_pad(total, n_seq);
   a.delta = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kWsHeader + seq_table_bytes(n_seq));
   a.lse2 = a.delta + (size_t)Hq * a.N_pad;
+  {
+    // long key tiles split by query range, planned on the device: flags, table, fp32 partials
+    int chunk;
+    const int cap = varlen_split_cap(p, total, Hq, Hkv, &chunk);
+    if (cap > 0) {
+      char* base = reinterpret_cast<char*>(a.lse2 + (size_t)Hq * a.N_pad);
+      base = reinterpret_cast<char*>(ws) + align_up((size_t)(base - reinterpret_cast<char*>(ws)), 256);
+      a.kv_chunk = chunk;
+      a.n_split = cap;
+      a.kv_bound = a.N_pad / 128;
+      a.kv_flag = reinterpret_cast<int32_t*>(base);
+      base += align_up((size_t)Hkv * a.kv_bound * sizeof(int32_t), 256);
+      a.kv_tab = reinterpret_cast<int4*>(base);
+      a.kv_part = reinterpret_cast<float*>(base + align_up((size_t)cap * sizeof(int4), 256));
+    }
+  }
   a.scale = scale_of(pat, d);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   if (!make_tmap_bf16(&a.tm_q, q.ptr, d, total, Hq, 1, q.stride_t, q.stride_h, q.stride_b, 128) ||

@@ -128,6 +128,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
   int j, g, b, kc = -1;  // kc >= 0: chunk kc of a split key tile
   if ((int)blockIdx.x < a.n_split) {
     const int4 e = a.kv_tab[blockIdx.x];
+    if (e.w < 0) return;  // an unused slot of a packed batch's table (whole CTA, before any barrier)
     j = e.x; g = e.y; b = e.z; kc = e.w;
   } else {
     const int x = (int)blockIdx.x - a.n_split;
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
   }
   // the rows of this CTA's sequence: [row0, row0 + N) of the token axis; statistics tiles from tile0
   int row0 = 0, N = a.N, tile0 = 0;
+  const int tg = j;  // the key tile on the packed token axis (a packed batch)
   if (a.varlen) {
     if (j >= a.seq_tab[a.n_seq]) return;  // whole CTA, before any barrier or TMEM use
     const int sq = seq_of_tile(a.seq_tab, a.n_seq, j);
@@ -149,7 +151,9 @@ __global__ void __launch_bounds__((4 * NP + 2) * 32, 1) bwd_dkdv_kernel(const __
   const Range iv = interval_of(a.pat, g);
   const Range rows = bwd_row_range(a.pat, iv, s0, s1, N);
   int i_lo = rows.lo / kTile, i_hi = (rows.hi + kTile - 1) / kTile;
-  if (a.kv_chunk > 0 && i_hi - i_lo > a.kv_chunk) {
+  const bool split = a.kv_chunk > 0 && (a.varlen ? a.kv_flag[(size_t)g * a.kv_bound + tg] != 0
+                                                 : i_hi - i_lo > a.kv_chunk);
+  if (split) {
     if (kc < 0) return;  // a split tile: its chunk CTAs do the work (before any barrier or TMEM use)
     i_lo += kc * a.kv_chunk;
     i_hi = imin(i_hi, i_lo + a.kv_chunk);
@@ -752,14 +756,64 @@ __global__ void __launch_bounds__(256) kv_split_table_kernel(Pat p, int N, int B
   }
 }
 
+// The chunk table of a packed batch (one block, after the sequence table): the same rule over
+// the packed key tiles of every sequence, within `cap` slots.  Tiles are taken in order while
+// their chunks fit; kv_flag marks the split ones, the rest stay whole; unused slots hold chunk -1.
+__global__ void __launch_bounds__(256) kv_split_table_varlen_kernel(Pat p, const int32_t* seq_tab, int n_seq, int Hkv,
+                                                                    int chunk, int cap, int bound, int4* tab,
+                                                                    int32_t* flag) {
+  __shared__ int offs[256];
+  const int tiles = seq_tab[n_seq], pairs = Hkv * tiles, t = threadIdx.x;
+  for (int i = t; i < cap; i += 256) tab[i] = make_int4(0, 0, 0, -1);
+  const int per = (pairs + 255) / 256;
+  const int lo = imin(pairs, t * per), hi = imin(pairs, lo + per);
+  auto range_of = [&](int q, int& g, int& tg) {
+    g = q / tiles;
+    tg = q % tiles;
+    const int sq = seq_of_tile(seq_tab, n_seq, tg);
+    return kv_range_tiles(p, interval_of(p, g), tg - seq_tab[sq], seq_tab[2 * n_seq + 1 + sq]);
+  };
+  int cnt = 0;
+  for (int q = lo; q < hi; ++q) {
+    int g, tg;
+    const int n = range_of(q, g, tg);
+    if (n > chunk) cnt += (n + chunk - 1) / chunk;
+  }
+  offs[t] = cnt;
+  __syncthreads();
+  if (t == 0) {
+    int acc = 0;
+    for (int i = 0; i < 256; ++i) { const int v = offs[i]; offs[i] = acc; acc += v; }
+  }
+  __syncthreads();  // also orders the sentinel fill before the entries below
+  int e = offs[t];
+  for (int q = lo; q < hi; ++q) {
+    int g, tg;
+    const int n = range_of(q, g, tg);
+    const int m = n > chunk ? (n + chunk - 1) / chunk : 0;
+    const bool fits = m > 0 && e + m <= cap;
+    flag[(size_t)g * bound + tg] = fits ? 1 : 0;
+    if (fits)
+      for (int k = 0; k < m; ++k) tab[e + k] = make_int4(tg, g, 0, k);
+    e += m;
+  }
+}
+
 // dk, dv of the split key tiles: the chunks' fp32 partials summed in chunk order (one block per
 // tile, run by the block of its first chunk), dk scaled, rounded to bf16.
 template <int D>
 __global__ void __launch_bounds__(256) kv_split_reduce_kernel(const __grid_constant__ BwdArgs a) {
   const int e0 = blockIdx.x;
   const int4 t = a.kv_tab[e0];
-  if (t.w != 0) return;
-  const int j = t.x, g = t.y, b = t.z;
+  if (t.w != 0) return;  // not a tile's first chunk (or an unused slot)
+  int j = t.x, row0 = 0, N = a.N;
+  const int g = t.y, b = t.z;
+  if (a.varlen) {  // the key tile's sequence on the packed token axis
+    const int sq = seq_of_tile(a.seq_tab, a.n_seq, j);
+    j -= a.seq_tab[sq];
+    row0 = a.seq_tab[a.n_seq + 1 + sq];
+    N = a.seq_tab[2 * a.n_seq + 1 + sq];
+  }
   int n = 1;  // the tile's chunks are consecutive entries
   while (e0 + n < a.n_split && a.kv_tab[e0 + n].w == n) ++n;
   const int s0 = j * kTile;
@@ -773,11 +827,11 @@ __global__ void __launch_bounds__(256) kv_split_reduce_kernel(const __grid_const
       sv.x += v.x; sv.y += v.y; sv.z += v.z; sv.w += v.w;
       sk.x += k.x; sk.y += k.y; sk.z += k.z; sk.w += k.w;
     }
-    if (s0 + r < a.N) {
-      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb + (int64_t)(s0 + r) * a.dv_st +
-                           g * a.dv_sh + c4 * 4;
-      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb + (int64_t)(s0 + r) * a.dk_st +
-                           g * a.dk_sh + c4 * 4;
+    if (s0 + r < N) {
+      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(a.dv) + b * a.dv_sb +
+                           ((int64_t)row0 + s0 + r) * a.dv_st + g * a.dv_sh + c4 * 4;
+      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(a.dk) + b * a.dk_sb +
+                           ((int64_t)row0 + s0 + r) * a.dk_st + g * a.dk_sh + c4 * 4;
       *reinterpret_cast<uint2*>(dvr) = make_uint2(ptx::pack_bf16(sv.x, sv.y), ptx::pack_bf16(sv.z, sv.w));
       *reinterpret_cast<uint2*>(dkr) = make_uint2(ptx::pack_bf16(sk.x * a.scale, sk.y * a.scale),
                                                   ptx::pack_bf16(sk.z * a.scale, sk.w * a.scale));
@@ -802,7 +856,11 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
     const long long n_kv = (long long)nq * a.Hkv * a.B + a.n_split;
     if (n_kv > 0x7fffffffLL) return cudaErrorInvalidValue;
     if (a.n_split > 0) {
-      kv_split_table_kernel<<<1, 256, 0, s>>>(a.pat, a.N, a.B, a.Hkv, a.kv_chunk, a.kv_tab);
+      if (a.varlen)
+        kv_split_table_varlen_kernel<<<1, 256, 0, s>>>(a.pat, a.seq_tab, a.n_seq, a.Hkv, a.kv_chunk, a.n_split,
+                                                       a.kv_bound, a.kv_tab, a.kv_flag);
+      else
+        kv_split_table_kernel<<<1, 256, 0, s>>>(a.pat, a.N, a.B, a.Hkv, a.kv_chunk, a.kv_tab);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     kdkdv<<<(unsigned)n_kv, (4 * NPK + 2) * 32, Geo::kSmemKV, s>>>(a);

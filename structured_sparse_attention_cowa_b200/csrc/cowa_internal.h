@@ -120,9 +120,14 @@ struct BwdArgs {
   // kv_chunk query tiles; each writes fp32 partial dV, dK ([2][128][d]) to kv_part + e*2*128*d,
   // and a reduction kernel sums a tile's chunks in chunk order.  The unsplit CTA of such a tile
   // leaves at once.  Packed batches do not split (kv_chunk = 0).
+  // A packed batch plans its split on the device (the host cannot see the lengths): n_split is
+  // then a capacity, unused table slots hold chunk -1, and kv_flag[g * kv_bound + packed tile]
+  // says which key tiles were split (a tile that does not fit the capacity stays whole).
   int kv_chunk, n_split;
   int4* kv_tab;
   float* kv_part;
+  int32_t* kv_flag;
+  int kv_bound;
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
 };
 struct KvSplit {

@@ -22,6 +22,9 @@ pytestmark = pytest.mark.gpu
     (10, 2, 128, cw.Pattern(32, 200, 1000, 2), [1, 127, 0, 128, 300, 1000]),   # group of 5, an empty sequence
     (8, 4, 128, cw.Pattern(0, 40, 500, 4), [129, 257, 64]),                     # no sink, group of 2
     (4, 2, 64, cw.Pattern(8, 30, 200, 2), [int(x) for x in np.random.default_rng(3).integers(1, 150, 64)]),  # 64 short
+    # one and two KV heads with long sequences: the long key tiles are split, planned on the device
+    (4, 1, 128, cw.Pattern(64, 256, 4096, 1), [4096, 5, 1500, 0, 700]),
+    (8, 2, 128, cw.Pattern(32, 128, 4096, 2), [3000, 1, 2000]),
 ])
 def test_bwd_varlen_packed_batch(cuda_device, Hq, Hkv, d, pat, lens):
     total = sum(lens)
