@@ -138,7 +138,9 @@ cowa_status cowa_fwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H
  * Inputs  q, k, v, o, lse as produced/consumed by cowa_fwd; dO [B, N, H_q, d] bf16.
  * Outputs dq [B, N, H_q, d], dk and dv [B, N, H_kv, d], bf16 (fp32 accumulation).
  * The workspace holds fp32 row statistics (Delta = rowsum(dO * O) and lse * log2(e) per
- * query row). */
+ * query row) and, when a call has few KV heads, the query-range split of its long dK/dV key
+ * tiles: a table of chunks and their fp32 partial dk, dv (128 KB per chunk at d = 128), summed in
+ * chunk order so that results stay deterministic.  The size depends on the pattern and shape. */
 size_t cowa_bwd_workspace_size(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d);
 cowa_status cowa_bwd(const cowa_pattern* pat, int B, int N, int H_q, int H_kv, int d,
                      cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o, const float* lse,
@@ -172,8 +174,9 @@ cowa_status cowa_bwd_stages(const cowa_pattern* pat, int B, int N, int H_q, int 
  * cu_seqlens: DEVICE int32 [n_seq + 1], non-decreasing from 0 to total.  The device clamps the
  * offsets so that sequences stay in order, disjoint and inside [0, total) (a malformed table
  * cannot reach memory outside the tensors; its sequences are then the clamped ones).
- * Workspace: cowa_bwd_varlen_workspace_size(pat, n_seq, total, ...).  Other errors as for
- * cowa_bwd. */
+ * Workspace: cowa_bwd_varlen_workspace_size(pat, n_seq, total, ...), including room for the
+ * key-tile split of the longest batch of `total` rows (the split is planned on the device from
+ * the actual lengths).  Other errors as for cowa_bwd. */
 size_t cowa_bwd_varlen_workspace_size(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d);
 cowa_status cowa_bwd_varlen(const cowa_pattern* pat, int n_seq, int total, int H_q, int H_kv, int d,
                             const int32_t* cu_seqlens, cowa_tensor q, cowa_tensor k, cowa_tensor v, cowa_tensor o,
