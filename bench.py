@@ -483,7 +483,12 @@ class TpRank:
             cp, cpd = pat.c(), dpat.c()
             ws = lambda n: torch.zeros(max(256, n), dtype=torch.uint8, device=dev)
             b["ws_f"] = ws(lib.cowa_fwd_workspace_size(ctypes.byref(cp), B, N, nq, nk, d))
-            b["ws_b"] = ws(lib.cowa_bwd_workspace_size(ctypes.byref(cp), B, N, nq, nk, d))
+            n_b = lib.cowa_bwd_workspace_size(ctypes.byref(cp), B, N, nq, nk, d)
+            b["ws_b"] = ws(n_b)
+            # a workspace larger than header + row statistics means the call splits its long key
+            # tiles: two more launches (the chunk table and the reduction of the partials)
+            stats = 256 + (2 * B * nq * ((N + 127) // 128 * 128) * 4 + 255) // 256 * 256
+            b["split"] = n_b > stats
             b["ws_d"] = ws(lib.cowa_decode_workspace_size(ctypes.byref(cpd), dc["B"], nq, nk, dc["d"], dc["T_cap"]))
             self.bufs.append(b)
 
@@ -506,7 +511,8 @@ class TpRank:
 
     @property
     def launches_per_step(self) -> int:
-        return 6 * len(self.bufs)  # per run: forward 1, backward 3, decode 2
+        # per run: forward 1, backward 3 (+ 2 when it splits long key tiles), decode 2
+        return sum(6 + (2 if b["split"] else 0) for b in self.bufs)
 
 
 def run_cowa_tp(args, world, rank, local):
