@@ -42,6 +42,10 @@
  *     it (COWA_ERR_TIMEOUT).
  *   - The library keeps no mutable global state on the call path; calls on
  *     different streams with different workspaces may run concurrently.
+ *   - cowa_fwd, cowa_bwd and cowa_decode never synchronise the host and allocate
+ *     nothing, so a step made of them can be captured in a CUDA graph on a
+ *     capturing stream and replayed (same bits as the calls made directly).
+ *     cowa_workspace_status synchronises and is not capturable.
  */
 #ifndef COWA_H
 #define COWA_H
