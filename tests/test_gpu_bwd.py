@@ -212,11 +212,13 @@ def test_bwd_long_128k(cuda_device):
                    [(0, [5, 128]), (3, [20000, 40001]), (7, [131071])], cuda_gen=True)
 
 
-def test_bwd_stages_on_two_streams_match_single_call(cuda_device):
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,pat", [
+    (1, 1500, 10, 2, 128, cw.Pattern(64, 200, 1500, 2)),
+    (1, 4096, 4, 1, 128, cw.Pattern(64, 256, 4096, 1)),   # the dK/dV stage splits its key tiles
+])
+def test_bwd_stages_on_two_streams_match_single_call(cuda_device, B, N, Hq, Hkv, d, pat):
     """The staged entry point: preprocess, then dK/dV and dQ on two streams that both wait for
     it, gives the same bits as one cowa_bwd call (the kernels are deterministic)."""
-    B, N, Hq, Hkv, d = 1, 1500, 10, 2, 128
-    pat = cw.Pattern(64, 200, 1500, 2)
     _, (q, k, v, do) = _inputs(B, N, Hq, Hkv, d, cuda_device, extra=9)
     o, lse = cw.cowa_fwd(q, k, v, pat)
     dq1, dk1, dv1 = cw.cowa_bwd(q, k, v, o, lse, do, pat)
