@@ -894,7 +894,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, int stages, cudaStream_t s) {
 KvSplit kv_split_plan(const Pat& p, int B, int N, int Hq, int Hkv) {
   constexpr long long kSms = 148;  // B200
   KvSplit sp{0, 0};
-  const int nq = (N + kTile - 1) / kTile, grp = Hq / Hkv;
+  const int nq = (N + kTile - 1) / kTile;
   long long total = 0;
   int longest = 0;
   for (int g = 0; g < Hkv; ++g) {
@@ -905,7 +905,7 @@ KvSplit kv_split_plan(const Pat& p, int B, int N, int Hq, int Hkv) {
       longest = imax(longest, n);
     }
   }
-  // query tiles per SM over the launch, each costing grp heads x 2 sub-steps alike
+  // query tiles per SM over the launch (each costs the same grp heads x 2 sub-steps everywhere)
   const long long per_sm = total * B / kSms;
   const int chunk = (int)(per_sm > 8 ? per_sm : 8);
   if (longest <= chunk) return sp;
@@ -918,7 +918,7 @@ KvSplit kv_split_plan(const Pat& p, int B, int N, int Hq, int Hkv) {
     }
   }
   sp.n_entries *= B;
-  (void)grp;
+  (void)Hq;  // every key tile walks its query tiles for all Hq / Hkv heads alike
   return sp;
 }
 
