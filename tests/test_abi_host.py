@@ -276,6 +276,26 @@ def test_bwd_workspace_holds_the_split_of_long_key_tiles():
     assert last == 256 + 2 * 5 * 32768 * 4 + 256 + 13 * 2 * 128 * 128 * 4
 
 
+def test_bwd_varlen_workspace_reserves_the_split_only_when_it_can_happen():
+    """A packed batch plans its key-tile split on the device, so its workspace reserves room as
+    for one sequence of all its rows: nothing for the 8-head 32K layer, table slots (twice that
+    plan's 121 chunks + 64), tile flags and partials for one KV head of it."""
+    L = cw.lib()
+
+    def ws(pat, n_seq, total, Hq, Hkv):
+        return L.cowa_bwd_varlen_workspace_size(ctypes.byref(pat.c()), n_seq, total, Hq, Hkv, 128)
+
+    n_seq, total = 3, 32768
+    rows = (total // 128 + n_seq) * 128
+    seq_tab = (3 * n_seq + 1) * 4
+    base = lambda Hq: 256 + (seq_tab + 255) // 256 * 256 + 2 * Hq * rows * 4
+    assert ws(cw.Pattern(128, 2048, 32768, 8), n_seq, total, 40, 8) == base(40)
+    cap = 2 * 121 + 64
+    flags = (1 * (rows // 128) * 4 + 255) // 256 * 256
+    one = ws(cw.Pattern(128, 2048, 32768, 8, kv_head_base=0, h_kv_global=8), n_seq, total, 5, 1)
+    assert one == base(5) + flags + (cap * 16 + 255) // 256 * 256 + cap * 2 * 128 * 128 * 4
+
+
 def test_compact_entry_points_reject_bad_arguments():
     L = cw.lib()
     p = cw.Pattern(20, 100, 2000, 2).c()
