@@ -515,6 +515,39 @@ class TpRank:
         return sum(6 + (2 if b["split"] else 0) for b in self.bufs)
 
 
+def tp_projection(P: int, order: str, steps: int, warmup: int, dev) -> dict:
+    """KV-head tensor parallelism projected on one GPU (a `parts` entry of the default line): the
+    P ranks' calls (the 32K layer's fwd + bwd and the 128K decode, split by KV head) run one rank
+    after another; with no exchange step each rank's time is the time it would take on its own
+    GPU, so the slowest rank's time is the P-GPU step."""
+    import torch
+
+    from structured_sparse_attention_cowa_b200 import cowa as cw
+    from structured_sparse_attention_cowa_b200 import synth
+
+    rank_ms = []
+    for r in range(P):
+        tr = TpRank(cw, synth, torch, dev, r, P, order)
+        for _ in range(warmup):
+            tr.fwd(); tr.bwd(); tr.dec()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            tr.fwd(); tr.bwd(); tr.dec()
+        b.record()
+        torch.cuda.synchronize()
+        bad = [x for x in tr.statuses() if x != 0]
+        if bad:
+            raise RuntimeError(f"device status {bad[0]} in the TP projection (rank {r})")
+        rank_ms.append(a.elapsed_time(b) / steps)
+        del tr
+        torch.cuda.empty_cache()
+    return {"P": P, "order": order, "projected_step_ms": max(rank_ms), "rank_ms": rank_ms,
+            "slowest_over_mean": max(rank_ms) / statistics.mean(rank_ms),
+            "note": "ranks run in turn on this GPU; the slowest rank's time is the P-GPU step"}
+
+
 def run_cowa_tp(args, world, rank, local):
     """--shard heads: the whole 32K layer and the whole 128K decode batch split by KV head over P
     ranks (strong scaling), each rank's calls over its own runs of global KV heads.  Under
@@ -978,6 +1011,7 @@ def run_cowa(args, world, rank, local):
     # ---- the other configurations, each kernel timed alone (burst peak), one GPU only
     if world == 1 and not args.no_parts:
         parts.update(config_parts(dev, kc, vc, burst, hbm, sweep=args.sweep))
+        parts["kv_head_tp4_projected"] = tp_projection(4, "folded", 3, 3, dev)
 
     if dist is not None:
         dist.destroy_process_group()
