@@ -1,6 +1,7 @@
 """Small, fixed invocations of each hot kernel for profiling with ncu.
 
-    python -m structured_sparse_attention_cowa_b200.profile_cases {fwd32k,bwd32k,decode128k_b4,decode128k_e4m3_b4,all}
+    python -m structured_sparse_attention_cowa_b200.profile_cases
+        {fwd32k,bwd32k,bwd32k_one_head,decode128k_b4,decode128k_e4m3_b4,all}
         [--reps R]
 
 Each case allocates its seeded inputs on cuda:0 (a few GB at most), calls the C ABI
@@ -57,6 +58,25 @@ def case_bwd32k(dev, reps):
     return wss
 
 
+def case_bwd32k_one_head(dev, reps):
+    """One KV head of the 32K layer (a rank of KV-head tensor parallelism: kv_head_base = 0,
+    h_kv_global = 8): the backward splits its long key tiles (121 chunks of 78 query tiles)."""
+    import ctypes
+
+    B, N, Hq, Hkv, d = 1, 32768, 5, 1, 128
+    q = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("q"), dev)
+    k = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("k"), dev)
+    v = synth.cuda_normal_bf16((B, N, Hkv, d), synth.seed_of("v"), dev)
+    do = synth.cuda_normal_bf16((B, N, Hq, d), synth.seed_of("do"), dev)
+    pat = cw.Pattern(128, 2048, 32768, 8, kv_head_base=0, h_kv_global=8)
+    o, lse = cw.cowa_fwd(q, k, v, pat)
+    n = cw.lib().cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, Hq, Hkv, d)
+    ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    for _ in range(reps):
+        cw.cowa_bwd(q, k, v, o, lse, do, pat, workspace=ws)
+    return [ws]
+
+
 def case_decode128k_b4(dev, reps):
     B, Hq, Hkv, d, Tc = 4, 40, 8, 128, 131072
     pat = cw.Pattern(128, 4096, 131072, 8)
@@ -90,8 +110,8 @@ def case_decode128k_e4m3_b4(dev, reps):
     return [ws]
 
 
-CASES = {"fwd32k": case_fwd32k, "bwd32k": case_bwd32k, "decode128k_b4": case_decode128k_b4,
-         "decode128k_e4m3_b4": case_decode128k_e4m3_b4}
+CASES = {"fwd32k": case_fwd32k, "bwd32k": case_bwd32k, "bwd32k_one_head": case_bwd32k_one_head,
+         "decode128k_b4": case_decode128k_b4, "decode128k_e4m3_b4": case_decode128k_e4m3_b4}
 
 
 def main(argv=None):
