@@ -276,6 +276,56 @@ def test_bwd_workspace_holds_the_split_of_long_key_tiles():
     assert last == 256 + 2 * 5 * 32768 * 4 + 256 + 13 * 2 * 128 * 128 * 4
 
 
+def _split_plan_bytes(S, L, T, D, H, G0, B, N, Hq, Hkv, d):
+    """The key-tile split rule restated from its description: a key tile's query range is every
+    query tile from its own to the end if its keys include sink or interval keys, else up to the
+    end of the band; chunks of (sum of ranges x B / 148) query tiles, at least 8, when the longest
+    range exceeds that; per chunk a 16-byte table entry and fp32 partial dV, dK."""
+    nq = (N + 127) // 128
+
+    def bound(i):
+        return S + (i * (T - S)) // H
+
+    total, ranges = 0, []
+    for g in range(Hkv):
+        slot = ((G0 + g) % D) * (H // D)
+        lo, hi = bound(slot), bound(slot + 1)
+        for j in range(nq):
+            s0, s1 = j * 128, min(N, j * 128 + 128)
+            special = s0 < S or (lo < hi and lo < s1 and hi > s0)
+            end = N if special else min(N, s1 - 1 + L)
+            n = (max(s0, end) + 127) // 128 - s0 // 128
+            ranges.append(n)
+            total += n
+    chunk = max(8, total * B // 148)
+    if max(ranges) <= chunk:
+        return 0
+    entries = B * sum((n + chunk - 1) // chunk for n in ranges if n > chunk)
+    return (entries * 16 + 255) // 256 * 256 + entries * 2 * 128 * d * 4
+
+
+def test_bwd_workspace_matches_the_split_rule_on_random_shapes():
+    L = cw.lib()
+    rng = np.random.default_rng(5)
+    for _ in range(60):
+        H = int(rng.choice([1, 2, 4, 8]))
+        D = int(rng.choice([x for x in (1, 2, 4, 8) if H % x == 0]))
+        Hkv = int(rng.integers(1, H + 1))
+        G0 = int(rng.integers(0, H - Hkv + 1))
+        grp = int(rng.choice([1, 2, 5, 8]))
+        B, d = int(rng.integers(1, 3)), int(rng.choice([64, 128]))
+        N = int(rng.integers(1, 6000))
+        S = int(rng.integers(0, 300))
+        T = S + int(rng.integers(0, 7000))
+        Lw = int(rng.choice([1, 64, 257, 2048, 2**31 - 1]))
+        pat = cw.Pattern(S, Lw, T, D, kv_head_base=G0, h_kv_global=H)
+        got = L.cowa_bwd_workspace_size(ctypes.byref(pat.c()), B, N, grp * Hkv, Hkv, d)
+        n_pad = (N + 127) // 128 * 128
+        want = 256 + (2 * B * grp * Hkv * n_pad * 4 + 255) // 256 * 256 + \
+            _split_plan_bytes(S, Lw, T, D, H, G0, B, N, grp * Hkv, Hkv, d)
+        assert got == want, (S, Lw, T, D, H, G0, B, N, grp, Hkv, d, got, want)
+
+
 def test_bwd_varlen_workspace_reserves_the_split_only_when_it_can_happen():
     """A packed batch plans its key-tile split on the device, so its workspace reserves room as
     for one sequence of all its rows: nothing for the 8-head 32K layer, table slots (twice that
